@@ -1,0 +1,80 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case below plants one mistake in a copy of the oracle's C source (on the
+CPU, in a temporary directory), builds it, points the oracle binding at it and
+runs the pin tests: at least one pin must fail for every mutant.
+"""
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "msa_oracle.c")
+
+MUTANTS = {
+    "rope_sign": ("x[i] = x0 * c - x1 * s;", "x[i] = x0 * c + x1 * s;"),
+    "rope_frequency": ("pow(theta, -2.0 * (double)i / (double)d)", "pow(theta, -1.0 * (double)i / (double)d)"),
+    "rope_pairing": ("double x0 = x[i], x1 = x[i + h];", "double x0 = x[i], x1 = x[(i + h + 1) % d];"),
+    "encode_global_position": ("int64_t p = q * chunk + u; /* document-local position */",
+                               "int64_t p = t0 + q * chunk + u;"),
+    "encode_full_chunk_divisor": ("kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)n);",
+                                  "kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)chunk);"),
+    "encode_norm_unrounded": ("double x = orc_bf16_to_double(b);", "double x = sr[(size_t)h * d + i] / (double)n + 1e-3;"),
+    "route_no_head_mean": ("double sc = cos_sum / (double)hr;", "double sc = cos_sum;"),
+    "route_mean_not_max": ("if (sc > best) best = sc;         /* max over rows and chunks */",
+                           "best = (best == -INFINITY ? 0.0 : best) + sc;"),
+    "route_missing_knorm": ("cos_sum += dot * inv_q[(size_t)t * hr + h] * inv_k[(size_t)c * hr + h];",
+                            "cos_sum += dot * inv_q[(size_t)t * hr + h];"),
+    "route_ties_high_id": ("return (x->id > y->id) - (x->id < y->id);", "return (x->id < y->id) - (x->id > y->id);"),
+    "route_transposed_head": ("kbar_r + ((size_t)c * hr + h) * d, d);", "kbar_r + ((size_t)c * hr + (hr - 1 - h)) * d, d);"),
+    "attend_gqa_modulo": ("int kh = h / group;", "int kh = h % hkv;"),
+    "attend_causal_strict": ("for (int64_t j = 0; j < n_loc && j <= g; ++j) {", "for (int64_t j = 0; j < n_loc && j < g; ++j) {"),
+    "attend_no_query_offset": ("orc_rope(qv, d, pos_offset + (double)g, rope_theta);", "orc_rope(qv, d, (double)g, rope_theta);"),
+    "attend_lse_no_max": ("lse[(size_t)r * hq + h] = mx + log(den);", "lse[(size_t)r * hq + h] = log(den);"),
+    "bf16_truncate": ("double r = nearbyint(ldexp(ax, -q));", "double r = floor(ldexp(ax, -q));"),
+    "gather_skips_last_chunk": ("for (int64_t c = doc_chunk_off[doc]; c < doc_chunk_off[doc + 1]; ++c) {",
+                                "for (int64_t c = doc_chunk_off[doc]; c + 1 < doc_chunk_off[doc + 1]; ++c) {"),
+}
+
+PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _build(src_text, workdir, name):
+    c = os.path.join(workdir, name + ".c")
+    so = os.path.join(workdir, name + ".so")
+    with open(c, "w") as f:
+        f.write(src_text)
+    shutil.copy(os.path.join(os.path.dirname(SRC), "msa_oracle.h"), workdir)
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-o", so, c,
+                    "-lm"], check=True)
+    return so
+
+
+def _failing_pins():
+    failed = []
+    for t in PIN_TESTS:
+        try:
+            t()
+        except Exception:  # any assertion or error counts as caught
+            failed.append(t.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    before, after = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(before) >= 1, f"mutation site for {name} not found"
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _build(text.replace(before, after, 1), tmp, name)
+        oracle.use_library(so)
+        try:
+            failed = _failing_pins()
+        finally:
+            oracle.use_library(None)
+    assert failed, f"no pin caught the planted mistake {name}"
