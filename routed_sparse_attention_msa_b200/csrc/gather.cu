@@ -1,0 +1,109 @@
+// Context assembly: the chunk list of each sequence's selected documents,
+// and (host content tier, device-pull mode) the copy of their pooled K/V rows
+// from mapped pinned host memory into a device staging buffer.
+//
+// ["MSA: Memory Sparse Attention", Inference Pipeline stage 2 — load only the
+// selected K-bar/V-bar and concatenate with local context; the Memory Parallel
+// paragraph — content K-bar/V-bar stays in host DRAM and is fetched when
+// selected; "MSA-arXiv26", 核心方法 / Memory Parallel inference (tiered storage)]
+#include "msa_internal.cuh"
+
+namespace msa {
+namespace {
+
+// One CTA: an exclusive scan over the (sequence, rank) pairs of the selected
+// documents' chunk counts gives each document's place in the list.
+__global__ void __launch_bounds__(1024) gather_index_kernel(
+    const int64_t* __restrict__ doc_chunk_off, const int32_t* __restrict__ top_ids, int n_seq,
+    int k, int64_t* __restrict__ sel_off, int64_t* __restrict__ sel_chunk) {
+  __shared__ int64_t warp_sums[32];
+  __shared__ int64_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int64_t n_pairs = (int64_t)n_seq * k;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n_pairs; base += blockDim.x) {
+    const int64_t p = base + tid;
+    int64_t c0 = 0, n = 0;
+    if (p < n_pairs) {
+      int32_t doc = top_ids[p];
+      c0 = doc_chunk_off[doc];
+      n = doc_chunk_off[doc + 1] - c0;
+    }
+    int64_t x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int64_t w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int64_t start = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + x - n;
+    if (p < n_pairs) {
+      for (int64_t i = 0; i < n; ++i) sel_chunk[start + i] = c0 + i;
+      if (p % k == 0) sel_off[p / k] = start;
+      if (p == n_pairs - 1) sel_off[n_seq] = start + n;
+    }
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = start + n;
+    __syncthreads();
+  }
+}
+
+// One warp per selected row: 2 x hkv x 256 B read from mapped host memory
+// with 16-byte loads, written to the staging buffers.
+__global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint16_t* __restrict__ vbar,
+                                   const int64_t* __restrict__ sel_total,
+                                   const int64_t* __restrict__ sel_chunk, int64_t cap, int hkv,
+                                   uint16_t* __restrict__ stage_k, uint16_t* __restrict__ stage_v) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = min(*sel_total, cap);
+  const int vecs = hkv * kHeadDim / 8;  // uint4 per row
+  for (int64_t j = gw; j < total; j += nw) {
+    const int64_t c = sel_chunk[j];
+    const uint4* sk = reinterpret_cast<const uint4*>(kbar + (size_t)c * hkv * kHeadDim);
+    const uint4* sv = reinterpret_cast<const uint4*>(vbar + (size_t)c * hkv * kHeadDim);
+    uint4* dk = reinterpret_cast<uint4*>(stage_k + (size_t)j * hkv * kHeadDim);
+    uint4* dv = reinterpret_cast<uint4*>(stage_v + (size_t)j * hkv * kHeadDim);
+    for (int i = lane; i < vecs; i += 32) {
+      uint4 a = sk[i];
+      uint4 b = sv[i];
+      dk[i] = a;
+      dv[i] = b;
+    }
+  }
+}
+
+}  // namespace
+
+msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
+                               int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st) {
+  gather_index_kernel<<<1, 1024, 0, st>>>(b.doc_chunk_off, top_ids, n_seq, k, sel_off, sel_chunk);
+  return launch_check("gather: chunk list");
+}
+
+msa_status launch_gather_pull(const msa_bank_layer& b, const int64_t* sel_off, const int64_t* sel_chunk,
+                              int64_t cap, uint16_t* stage_k, uint16_t* stage_v, cudaStream_t st) {
+  int64_t warps = cap;
+  int64_t blocks = (warps * 32 + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks < 1) blocks = 1;
+  // sel_off[n_seq] is the total row count; the caller passes its address.
+  gather_pull_kernel<<<(unsigned)blocks, 256, 0, st>>>(b.kbar, b.vbar, sel_off, sel_chunk, cap, b.hkv,
+                                                       stage_k, stage_v);
+  return launch_check("gather: device pull from host memory");
+}
+
+}  // namespace msa

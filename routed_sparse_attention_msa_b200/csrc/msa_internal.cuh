@@ -1,0 +1,103 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// ---------------------------------------------------------------- errors
+msa_status fail(msa_status s, const char* fmt, ...);
+msa_status cuda_fail(cudaError_t e, const char* what);
+msa_status launch_check(const char* what);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxSeq = 256;
+
+// ------------------------------------------------------- small device math
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ float bf1(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// fp32 -> bf16, round to nearest even (NaN kept quiet).
+__device__ __forceinline__ uint32_t f2bf_bits(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0x7FC0u;
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return u >> 16;
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  return f2bf_bits(lo) | (f2bf_bits(hi) << 16);
+}
+
+// Order-preserving map of fp32 to uint32 (larger float -> larger integer).
+// 0 is below every encoded value and marks "no score".
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__host__ __device__ __forceinline__ float unord_f32(uint32_t o) {
+  if (o == 0u) return -INFINITY;
+  uint32_t u = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float f;
+  __builtin_memcpy(&f, &u, 4);
+  return f;
+#endif
+}
+
+// ------------------------------------------------------------ host launchers
+
+// encode.cu
+msa_status launch_encode(const msa_encode_args& a, cudaStream_t st);
+msa_status launch_bank_norms(const uint16_t* kbar_r, int64_t n_chunks, int hr, float eps,
+                             float* inv_norm, cudaStream_t st);
+
+// Routing plan shared by the scoring kernels: the query rows of one call,
+// their sequences, and the workspace pieces.
+struct RoutePlan {
+  const uint16_t* qr;          // [T, hr, d]
+  const float* kr_inv_norm;    // [C, hr]
+  const int32_t* chunk_doc;    // [C]
+  const uint16_t* kbar_r;      // [C, hr, d]
+  int64_t n_chunks, n_docs;
+  int32_t hr, n_rows, n_seq;
+  int32_t q_seq_off[kMaxSeq + 1];
+  float* invq;                 // ws [T, hr]: 1 / (hr * max(||q||, eps))
+  uint32_t* doc_key;           // ws [S, D]: ordered doc scores (0 = none)
+};
+
+// score.cu
+msa_status launch_qprep(const RoutePlan& p, float eps, cudaStream_t st);
+msa_status launch_score_simt(const RoutePlan& p, cudaStream_t st);
+// score_tc.cu
+msa_status launch_score_tc(const RoutePlan& p, cudaStream_t st);
+bool score_tc_supported(const RoutePlan& p);
+bool score_tc_built();
+int tc_error_take();  // 1 if a tensor-core kernel's bounded wait ran out since the last call
+
+// topk.cu
+size_t topk_workspace(int n_seq, int64_t n_docs, int k);
+msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k,
+                       int32_t* top_ids, float* top_scores, float* all_scores, void* ws,
+                       cudaStream_t st);
+
+// gather.cu
+msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
+                               int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st);
+msa_status launch_gather_pull(const msa_bank_layer& b, const int64_t* sel_off,
+                              const int64_t* sel_chunk, int64_t cap, uint16_t* stage_k,
+                              uint16_t* stage_v, cudaStream_t st);
+
+// attend.cu
+size_t attend_workspace(const msa_attend_args& a, int* n_splits_out);
+msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,221 @@
+// Top-k documents per sequence from the per-document routing scores.
+//
+// ["MSA: Memory Sparse Attention", Overall Design: Architecture — selects the
+// Top-k documents; "MSA-arXiv26", 核心方法 — cosine similarity, top-k documents]
+//
+// Every document gets a 64-bit key: the order-preserving encoding of its
+// score in the high word and (0xFFFFFFFF - id) in the low word, so the total
+// order "score descending, then id ascending" is plain unsigned comparison
+// and all keys are distinct. A document that was never scored (no chunks)
+// has score word 0, below every real score.
+//
+// k <= 32: each warp keeps its best k keys sorted across lanes; a batch of 32
+// new keys is filtered against the k-th key with one ballot and the few
+// survivors are inserted by shuffles. CTAs take slices of the documents; the
+// last CTA of a sequence to finish (atomic ticket, no waiting) merges the
+// slices' candidates. k > 32: one CTA per sequence runs an 8-pass radix select
+// on the keys, collects the k keys at or above the k-th and sorts them.
+#include "msa_internal.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kDocsPerWarp = 512;
+constexpr int kDocsPerCta = kWarps * kDocsPerWarp;
+
+__device__ __forceinline__ uint64_t doc_key64(uint32_t score_key, int64_t doc) {
+  return ((uint64_t)score_key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)doc);
+}
+
+// Insert this lane's candidate `key` into the warp's sorted list (lane i holds
+// the i-th largest, i < k; lanes >= k are unused). Keys are distinct.
+__device__ __forceinline__ void warp_insert(uint64_t& list, uint64_t key, int k, int lane) {
+  uint64_t thr = __shfl_sync(0xffffffffu, list, k - 1);
+  unsigned m = __ballot_sync(0xffffffffu, key > thr);
+  while (m) {
+    int src = __ffs(m) - 1;
+    uint64_t v = __shfl_sync(0xffffffffu, key, src);
+    unsigned gt = __ballot_sync(0xffffffffu, lane < k && list > v);
+    int pos = __popc(gt);
+    uint64_t up = __shfl_up_sync(0xffffffffu, list, 1);
+    if (lane < k) {
+      if (lane == pos) list = v;
+      else if (lane > pos) list = up;
+    }
+    thr = __shfl_sync(0xffffffffu, list, k - 1);
+    m &= ~(1u << src);
+    m &= __ballot_sync(0xffffffffu, key > thr);
+  }
+}
+
+__device__ __forceinline__ void write_result(uint64_t key, int32_t* ids, float* scores) {
+  *ids = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+  *scores = unord_f32((uint32_t)(key >> 32));
+}
+
+__global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(
+    const uint32_t* __restrict__ doc_key, int64_t n_docs, int k, uint64_t* __restrict__ cand,
+    unsigned* __restrict__ tickets, int32_t* __restrict__ top_ids, float* __restrict__ top_scores,
+    float* __restrict__ all_scores) {
+  __shared__ uint64_t s_lists[kWarps][32];
+  __shared__ bool s_last;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int s = blockIdx.y;
+  const int part = blockIdx.x;
+  const int n_parts = gridDim.x;
+  const uint32_t* keys = doc_key + (size_t)s * n_docs;
+
+  uint64_t list = 0;
+  const int64_t w0 = (int64_t)part * kDocsPerCta + (int64_t)wid * kDocsPerWarp;
+  for (int it = 0; it < kDocsPerWarp / 32; ++it) {
+    int64_t doc = w0 + it * 32 + lane;
+    uint64_t key = 0;
+    if (doc < n_docs) {
+      uint32_t sk = keys[doc];
+      key = doc_key64(sk, doc);
+      if (all_scores) all_scores[(size_t)s * n_docs + doc] = unord_f32(sk);
+    }
+    warp_insert(list, key, k, lane);
+  }
+  s_lists[wid][lane] = list;
+  __syncthreads();
+  if (wid == 0) {
+    uint64_t merged = s_lists[0][lane];
+    for (int w = 1; w < kWarps; ++w) warp_insert(merged, lane < k ? s_lists[w][lane] : 0ull, k, lane);
+    if (lane < k) cand[((size_t)s * n_parts + part) * k + lane] = merged;
+    __threadfence();
+    unsigned t = 0;
+    if (lane == 0) t = atomicAdd(tickets + s, 1u);
+    t = __shfl_sync(0xffffffffu, t, 0);
+    s_last = (t == (unsigned)(n_parts - 1));
+  }
+  __syncthreads();
+  if (!s_last || wid != 0) return;
+  __threadfence();
+  uint64_t fin = 0;
+  const uint64_t* c = cand + (size_t)s * n_parts * k;
+  for (int64_t i0 = 0; i0 < (int64_t)n_parts * k; i0 += 32) {
+    int64_t i = i0 + lane;
+    uint64_t key = i < (int64_t)n_parts * k ? __ldcg(c + i) : 0ull;
+    warp_insert(fin, key, k, lane);
+  }
+  const int kk = k < n_docs ? k : (int)n_docs;
+  if (lane < kk) write_result(fin, top_ids + (size_t)s * kk + lane, top_scores + (size_t)s * kk + lane);
+  if (lane == 0) tickets[s] = 0u;  // ready for the next call
+}
+
+// Generic path: one CTA (1024 threads) per sequence.
+__global__ void __launch_bounds__(1024) topk_radix_kernel(
+    const uint32_t* __restrict__ doc_key, int64_t n_docs, int k, int32_t* __restrict__ top_ids,
+    float* __restrict__ top_scores, float* __restrict__ all_scores) {
+  extern __shared__ uint64_t s_sel[];  // [pow2 >= k]
+  __shared__ unsigned s_hist[256];
+  __shared__ uint64_t s_prefix, s_mask;
+  __shared__ int s_krem;
+  __shared__ unsigned s_count;
+  const int s = blockIdx.x;
+  const uint32_t* keys = doc_key + (size_t)s * n_docs;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_prefix = 0;
+    s_mask = 0;
+    s_krem = k;
+    s_count = 0;
+  }
+  if (all_scores)
+    for (int64_t j = tid; j < n_docs; j += blockDim.x) all_scores[(size_t)s * n_docs + j] = unord_f32(keys[j]);
+  __syncthreads();
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
+    __syncthreads();
+    const uint64_t pre = s_prefix, msk = s_mask;
+    for (int64_t j = tid; j < n_docs; j += blockDim.x) {
+      uint64_t key = doc_key64(keys[j], j);
+      if ((key & msk) == pre) atomicAdd(&s_hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int krem = s_krem;
+      unsigned cum = 0;
+      int b = 255;
+      for (; b > 0; --b) {
+        if ((int)(cum + s_hist[b]) >= krem) break;
+        cum += s_hist[b];
+      }
+      s_krem = krem - (int)cum;
+      s_prefix = pre | ((uint64_t)b << shift);
+      s_mask = msk | (0xFFull << shift);
+    }
+    __syncthreads();
+  }
+  const uint64_t kth = s_prefix;  // the k-th largest key (keys are distinct)
+  int pow2 = 1;
+  while (pow2 < k) pow2 <<= 1;
+  for (int i = tid; i < pow2; i += blockDim.x) s_sel[i] = 0;
+  __syncthreads();
+  for (int64_t j = tid; j < n_docs; j += blockDim.x) {
+    uint64_t key = doc_key64(keys[j], j);
+    if (key >= kth) {
+      unsigned p = atomicAdd(&s_count, 1u);
+      if (p < (unsigned)k) s_sel[p] = key;
+    }
+  }
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < pow2; i += blockDim.x) {
+        int j = i ^ stride;
+        if (j > i) {
+          bool desc = (i & size) == 0;
+          uint64_t a = s_sel[i], b = s_sel[j];
+          if (desc ? (a < b) : (a > b)) {
+            s_sel[i] = b;
+            s_sel[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < k; i += blockDim.x)
+    write_result(s_sel[i], top_ids + (size_t)s * k + i, top_scores + (size_t)s * k + i);
+}
+
+}  // namespace
+
+size_t topk_workspace(int n_seq, int64_t n_docs, int k) {
+  int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;
+  if (k > 32) return 256;
+  return align_up((size_t)n_seq * parts * k * sizeof(uint64_t), 256) +
+         align_up((size_t)n_seq * sizeof(unsigned), 256);
+}
+
+// ws must be zero-initialised once (the tickets reset themselves).
+msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k, int32_t* top_ids,
+                       float* top_scores, float* all_scores, void* ws, cudaStream_t st) {
+  if (k > n_docs) k = (int)n_docs;
+  if (k <= 32) {
+    int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;
+    uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
+    unsigned* tickets = reinterpret_cast<unsigned*>(
+        reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * k * sizeof(uint64_t), 256));
+    dim3 grid((unsigned)parts, (unsigned)n_seq);
+    topk_warp_kernel<<<grid, kWarps * 32, 0, st>>>(doc_key, n_docs, k, cand, tickets, top_ids,
+                                                   top_scores, all_scores);
+    return launch_check("route: top-k (warp)");
+  }
+  int pow2 = 1;
+  while (pow2 < k) pow2 <<= 1;
+  size_t smem = (size_t)pow2 * sizeof(uint64_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "route: top-k shared memory");
+  }
+  topk_radix_kernel<<<n_seq, 1024, smem, st>>>(doc_key, n_docs, k, top_ids, top_scores, all_scores);
+  return launch_check("route: top-k (radix)");
+}
+
+}  // namespace msa
