@@ -1,0 +1,652 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA routed decode step on B200.
+
+One step = for every routing layer of the workload: route the step's query
+routing rows against the layer's whole pooled routing-key bank (score + top-k),
+gather the selected documents' pooled K/V (from pinned host memory for the
+100M-token workload), and attend over them plus the local K/V. Inputs are
+seeded synthetic tensors shaped like the pages' memory banks (the datasets the
+pages evaluate on are not used).
+
+Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead
+(the only other place this script runs oracle code, besides the cpu_baseline
+leg of the default arm).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
+    p.add_argument("--score-kernel", choices=["auto", "simt", "tc"], default="auto")
+    p.add_argument("--gather", choices=["copy", "pull"], default="pull",
+                   help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
+    p.add_argument("--content-layers", type=int, default=1,
+                   help="host-tier content banks to allocate; layer l uses bank l mod this (0: one per layer "
+                        "if host RAM allows)")
+    p.add_argument("--layers", type=int, default=0, help="override the workload's layer count (0: as defined)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile-steps", type=int, default=0,
+                   help="only run warmup + this many steps, no extra legs (for ncu captures)")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_for(kernel: str, src: str, workload: str, bytes_scale: float = 1.0):
+    """DRAM bytes per launch from a committed ncu summary, or None if the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e:
+        return None
+    h = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+    if e.get("source_sha") != h:
+        return None
+    return float(e["bytes_per_launch"]) * bytes_scale
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(dev: int) -> str:
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return str(dev)
+
+
+# --------------------------------------------------------- workload engine
+
+class Routed:
+    """Device state and one routed decode step over all layers of a workload."""
+
+    def __init__(self, w: synth.Workload, args, dev: int):
+        import torch
+        import routed_sparse_attention_msa_b200 as msa
+        self.torch, self.msa, self.w, self.args = torch, msa, w, args
+        self.dev = dev
+        self.L = args.layers or w.n_layers
+        st = torch.cuda.current_stream().cuda_stream
+        self.dco, cdoc = w.index()
+        self.C = int(self.dco[-1])
+        self.max_doc_chunks = int(np.diff(self.dco).max())
+        self.dco_d = torch.from_numpy(self.dco).cuda()
+        self.cdoc_d = torch.from_numpy(cdoc).cuda()
+        S, k = w.n_seq, w.top_k
+        self.S, self.k = S, k
+        hr, hkv, d = w.hr, w.hkv, w.d
+
+        def dev_normal(shape, tid):
+            t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+            synth.normal_bf16_device(t.data_ptr(), t.numel(), tid, stream=st)
+            return t
+
+        # routing-key banks, one per layer, resident in HBM
+        self.kbar_r, self.inv = [], []
+        for l in range(self.L):
+            kr = dev_normal((self.C, hr, d), synth.tid("kbar_r", l))
+            iv = torch.empty((self.C, hr), dtype=torch.float32, device="cuda")
+            msa.bank_norms(kr, iv)
+            self.kbar_r.append(kr)
+            self.inv.append(iv)
+        # content banks: HBM, or pinned host memory for the host-tier workload
+        self.on_host = w.content_on_host
+        self.kbar, self.vbar = [], []
+        if self.on_host:
+            n_content = args.content_layers or self._host_content_layers()
+            for l in range(n_content):
+                for lst, kind in ((self.kbar, "kbar"), (self.vbar, "vbar")):
+                    h = torch.empty((self.C, hkv, d), dtype=torch.bfloat16, pin_memory=True)
+                    synth.normal_bf16_host_into(h.data_ptr(), h.numel(), synth.tid(kind, l))
+                    lst.append(h)
+        else:
+            n_content = self.L
+            for l in range(self.L):
+                self.kbar.append(dev_normal((self.C, hkv, d), synth.tid("kbar", l)))
+                self.vbar.append(dev_normal((self.C, hkv, d), synth.tid("vbar", l)))
+        self.n_content = n_content
+        self.banks = [msa.BankLayer(self.dco_d, self.cdoc_d, self.kbar_r[l], self.inv[l],
+                                    self.kbar[l % n_content], self.vbar[l % n_content], self.on_host,
+                                    self.max_doc_chunks) for l in range(self.L)]
+        # per-layer query routing rows with planted documents (built on the host)
+        rows = [w.route_rows] * S
+        self.T = sum(rows)
+        self.qr_h, self.plans = [], []
+        for l in range(self.L):
+            def key_rows(c, l=l):
+                return synth.bits_to_f64(synth.normal_bf16_host(hr * d, synth.tid("kbar_r", l), index0=c * hr * d)
+                                         ).reshape(hr, d)
+            qr, qso, plan = synth.make_routing_queries(key_rows, self.dco, rows, k, w.n_needles, hr, d, l)
+            self.qr_h.append(qr)
+            self.plans.append(plan)
+        self.qso = qso
+        # attention inputs: one decoded row per sequence over loc_len local tokens
+        self.Tq = S * w.attn_rows
+        self.Lloc = w.loc_len
+        self.q_seq_off = np.arange(S + 1, dtype=np.int32) * w.attn_rows
+        self.q_start = np.full(S, self.Lloc - w.attn_rows, np.int32)
+        self.loc_off = np.arange(S + 1, dtype=np.int32) * self.Lloc
+        self.q_h, self.kl_h, self.vl_h = [], [], []
+        for l in range(self.L):
+            self.q_h.append(synth.normal_bf16_host(self.Tq * w.hq * d, synth.tid("q_att", l)).reshape(self.Tq, w.hq, d))
+            self.kl_h.append(synth.normal_bf16_host(S * self.Lloc * hkv * d, synth.tid("k_loc", l)).reshape(
+                S * self.Lloc, hkv, d))
+            self.vl_h.append(synth.normal_bf16_host(S * self.Lloc * hkv * d, synth.tid("v_loc", l)).reshape(
+                S * self.Lloc, hkv, d))
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+        self.qr_d = [up(a) for a in self.qr_h]
+        self.q_d = [up(a) for a in self.q_h]
+        self.kl_d = [up(a) for a in self.kl_h]
+        self.vl_d = [up(a) for a in self.vl_h]
+        # outputs and workspaces (shared by layers; the stream orders their reuse)
+        kk = min(k, w.n_docs)
+        self.kk = kk
+        self.ids = [torch.empty((S, kk), dtype=torch.int32, device="cuda") for _ in range(self.L)]
+        self.scores = [torch.empty((S, kk), dtype=torch.float32, device="cuda") for _ in range(self.L)]
+        self.ws_route = torch.empty(msa.route_workspace(self.banks[0], S, self.T, k), dtype=torch.uint8, device="cuda")
+        self.cap = S * kk * self.max_doc_chunks
+        self.sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+        self.sel = torch.empty(self.cap, dtype=torch.int64, device="cuda")
+        if self.on_host:
+            self.stage_k = torch.empty((self.cap, hkv, d), dtype=torch.bfloat16, device="cuda")
+            self.stage_v = torch.empty((self.cap, hkv, d), dtype=torch.bfloat16, device="cuda")
+            self.ids_host = torch.empty(S * kk, dtype=torch.int32).pin_memory()
+            self.copy_stream = torch.cuda.Stream()
+            self.copy_done = torch.cuda.Event()
+            self.copy_done.record(self.copy_stream)
+        self.out = [torch.empty((self.Tq, w.hq, d), dtype=torch.bfloat16, device="cuda") for _ in range(self.L)]
+        self.pos_offset = float(k)
+        a0 = self._attend_args(0)
+        self.ws_attend = torch.empty(msa.attend_workspace(*a0, pos_offset=self.pos_offset, rope_theta=w.rope_theta),
+                                     dtype=torch.uint8, device="cuda")
+        self.mode = msa.GATHER_DEVICE_PULL if args.gather == "pull" else msa.GATHER_COPY_ENGINE
+        torch.cuda.synchronize()
+
+    def _host_content_layers(self) -> int:
+        need = 2 * self.C * self.w.hkv * self.w.d * 2 * self.L
+        try:
+            avail = os.sysconf("SC_AVPHYS_PAGES") * os.sysconf("SC_PAGE_SIZE")
+        except (ValueError, OSError):
+            avail = 0
+        return self.L if need < 0.6 * avail else 1
+
+    def _attend_args(self, l):
+        if self.on_host:
+            mk, mv, sel = self.stage_k, self.stage_v, None
+        else:
+            mk, mv, sel = self.banks[l].kbar, self.banks[l].vbar, self.sel
+        return (self.q_d[l], self.q_seq_off, self.q_start, self.kl_d[l], self.vl_d[l], self.loc_off, mk, mv,
+                self.sel_off, sel, self.cap)
+
+    def layer(self, l, ev=None):
+        msa = self.msa
+        if ev is not None:
+            msa.score_events(ev[0], ev[1])
+        msa.route(self.banks[l], self.qr_d[l], self.qso, self.k, self.ids[l], self.scores[l], self.ws_route,
+                  eps=self.w.eps)
+        if self.on_host:
+            msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel, self.stage_k, self.stage_v,
+                       mode=self.mode, doc_chunk_off_host=self.dco, top_ids_host=self.ids_host,
+                       copy_stream=self.copy_stream, done_event=self.copy_done)
+        else:
+            msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel)
+        msa.attend(*self._attend_args(l), self.out[l], self.ws_attend, pos_offset=self.pos_offset,
+                   rope_theta=self.w.rope_theta)
+
+    def step(self, evs=None):
+        for l in range(self.L):
+            self.layer(l, None if evs is None else evs[l])
+
+    def units_per_step(self) -> float:
+        return float(self.w.memory_tokens) * self.S * self.L
+
+    def score_bytes_per_launch(self) -> float:
+        w = self.w
+        return self.C * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+
+    def check_planted(self):
+        """Every layer's routed set must be its planted set (a property of the inputs)."""
+        bad = 0
+        for l in range(self.L):
+            got = self.ids[l].cpu().numpy()
+            for s in range(self.S):
+                if set(got[s].tolist()) != set(self.plans[l].docs[s]):
+                    bad += 1
+        return bad
+
+
+class Encode:
+    """Offline encode of the 10M-token corpus, once per layer over the same resident input."""
+
+    def __init__(self, w: synth.Workload, args, dev: int):
+        import torch
+        import routed_sparse_attention_msa_b200 as msa
+        self.torch, self.msa, self.w = torch, msa, w
+        self.L = args.layers or w.n_layers
+        st = torch.cuda.current_stream().cuda_stream
+        n = w.memory_tokens
+        self.inp = []
+        for kind, heads in (("k_tok", w.hkv), ("v_tok", w.hkv), ("kr_tok", w.hr)):
+            t = torch.empty((n, heads, w.d), dtype=torch.bfloat16, device="cuda")
+            synth.normal_bf16_device(t.data_ptr(), t.numel(), synth.tid(kind, 0), stream=st)
+            self.inp.append(t)
+        self.off_d = torch.from_numpy(w.doc_tok_off).cuda()
+        self.C, _, _ = msa.encode_plan(w.doc_tok_off, w.chunk)
+        C = self.C
+        self.out = dict(kbar=torch.empty((C, w.hkv, w.d), dtype=torch.bfloat16, device="cuda"),
+                        vbar=torch.empty((C, w.hkv, w.d), dtype=torch.bfloat16, device="cuda"),
+                        kbar_r=torch.empty((C, w.hr, w.d), dtype=torch.bfloat16, device="cuda"),
+                        kr_inv_norm=torch.empty((C, w.hr), dtype=torch.float32, device="cuda"),
+                        doc_chunk_off=torch.empty(w.n_docs + 1, dtype=torch.int64, device="cuda"),
+                        chunk_doc=torch.empty(C, dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+
+    def step(self, evs=None):
+        for l in range(self.L):
+            if evs is not None:
+                evs[l][0].record()
+            self.msa.encode(*self.inp, self.off_d, self.C, self.out, chunk=self.w.chunk,
+                            rope_theta=self.w.rope_theta, eps=self.w.eps)
+            if evs is not None:
+                evs[l][1].record()
+
+    def units_per_step(self):
+        return float(self.w.memory_tokens) * self.L
+
+    def kernel_bytes_per_launch(self):
+        w = self.w
+        return w.memory_tokens * (2 * w.hkv + w.hr) * w.d * 2 + self.C * ((2 * w.hkv + w.hr) * w.d * 2 + w.hr * 4 + 4)
+
+
+# ----------------------------------------------------------- CPU baseline
+
+def cpu_baseline(w: synth.Workload, max_chunks: int | None = None, layer: int = 0):
+    """The oracle, as it stands (single-threaded C), on one layer of the workload
+    (or a contiguous slice of it): route + gather + attend. Returns a dict."""
+    import oracle
+    dco, _ = w.index()
+    D = dco.size - 1
+    if max_chunks is not None and dco[-1] > max_chunks:
+        n_docs = int(np.searchsorted(dco, max_chunks, side="right") - 1)
+        dco = dco[: n_docs + 1]
+    C = int(dco[-1])
+    n_tok = int(w.doc_tok_off[dco.size - 1])
+    kr = synth.normal_bf16_host(C * w.hr * w.d, synth.tid("kbar_r", layer)).reshape(C, w.hr, w.d)
+    rows = [w.route_rows] * w.n_seq
+    qr, qso, plan = synth.make_routing_queries(lambda c: synth.bits_to_f64(kr[c]), dco, rows, w.top_k,
+                                               w.n_needles, w.hr, w.d, layer)
+    t0 = time.perf_counter()
+    ids, sc, _ = oracle.route(kr, dco, qr, qso, w.top_k, want_scores=False)
+    t_route = time.perf_counter() - t0
+    so, sel = oracle.gather(ids, dco)
+    kh = synth.normal_bf16_host(C * w.hkv * w.d, synth.tid("kbar", layer)).reshape(C, w.hkv, w.d)
+    vh = synth.normal_bf16_host(C * w.hkv * w.d, synth.tid("vbar", layer)).reshape(C, w.hkv, w.d)
+    S, L = w.n_seq, w.loc_len
+    q = synth.normal_bf16_host(S * w.attn_rows * w.hq * w.d, synth.tid("q_att", layer)).reshape(-1, w.hq, w.d)
+    kl = synth.normal_bf16_host(S * L * w.hkv * w.d, synth.tid("k_loc", layer)).reshape(-1, w.hkv, w.d)
+    vl = synth.normal_bf16_host(S * L * w.hkv * w.d, synth.tid("v_loc", layer)).reshape(-1, w.hkv, w.d)
+    t1 = time.perf_counter()
+    oracle.attend(q, np.arange(S + 1) * w.attn_rows, np.full(S, L - w.attn_rows), kl, vl, np.arange(S + 1) * L,
+                  kh, vh, so, sel, pos_offset=float(w.top_k))
+    t_att = time.perf_counter() - t1
+    total = t_route + t_att
+    return dict(tokens=n_tok * S, seconds=total, route_s=t_route, attend_s=t_att, chunks=C, docs=dco.size - 1,
+                layer_chunks=int(w.index()[0][-1]), full_docs=D)
+
+
+def encode_cpu_baseline(w: synth.Workload, n_docs: int = 2):
+    import oracle
+    off = w.doc_tok_off[: n_docs + 1]
+    n = int(off[-1])
+    k = synth.normal_bf16_host(n * w.hkv * w.d, synth.tid("k_tok", 0)).reshape(n, w.hkv, w.d)
+    v = synth.normal_bf16_host(n * w.hkv * w.d, synth.tid("v_tok", 0)).reshape(n, w.hkv, w.d)
+    r = synth.normal_bf16_host(n * w.hr * w.d, synth.tid("kr_tok", 0)).reshape(n, w.hr, w.d)
+    t0 = time.perf_counter()
+    oracle.encode(k, v, r, off, chunk=w.chunk, rope_theta=w.rope_theta, eps=w.eps)
+    return dict(tokens=n, seconds=time.perf_counter() - t0)
+
+
+# ---------------------------------------------------------------- arms
+
+def metric_of(name):
+    if name == "encode":
+        return "memory tokens encoded/s", "tokens/s"
+    return "memory tokens routed/s", "tokens/s"
+
+
+def config_of(w, eng, args, extra=None):
+    cfg = {"workload": w.name, "memory_tokens": w.memory_tokens, "docs": w.n_docs,
+           "layers": (args.layers or w.n_layers), "chunk": w.chunk, "hr": w.hr, "d": w.d}
+    if w.name != "encode":
+        cfg.update({"chunks_per_layer": eng.C, "sequences": w.n_seq, "routing_rows_per_seq": w.route_rows,
+                    "top_k": w.top_k, "hq": w.hq, "hkv": w.hkv, "local_tokens": w.loc_len,
+                    "content": "pinned_host" if w.content_on_host else "hbm",
+                    "gather": args.gather if w.content_on_host else "hbm_index",
+                    "score_kernel": args.score_kernel})
+    else:
+        cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
+    cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.workload(args.workload)
+    metric, unit = metric_of(w.name)
+    times = []
+    if w.name == "encode":
+        for i in range(args.warmup + args.steps):
+            r = encode_cpu_baseline(w, n_docs=1)
+            if i >= args.warmup:
+                times.append((r["tokens"], r["seconds"]))
+        sample = "1 document of 4096 tokens, one layer (oracle encode, single thread)"
+    else:
+        dco, _ = w.index()
+        cap = min(int(dco[-1]), 24_000)
+        for i in range(args.warmup + args.steps):
+            r = cpu_baseline(w, max_chunks=cap, layer=i % w.n_layers)
+            if i >= args.warmup:
+                times.append((r["tokens"], r["seconds"]))
+        sample = (f"one layer per step over the first {r['docs']} documents ({r['chunks']} of "
+                  f"{r['layer_chunks']} chunks): route + gather + attend, oracle single thread")
+    tok = sum(t for t, _ in times)
+    sec = sum(s for _, s in times)
+    value = tok / sec
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, None if w.name == "encode" else _Shape(w), args),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+class _Shape:
+    def __init__(self, w):
+        self.C = int(w.index()[0][-1])
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    import routed_sparse_attention_msa_b200 as msa
+    msa.set_score_kernel(args.score_kernel)
+    w = synth.workload(args.workload)
+    metric, unit = metric_of(w.name)
+    eng = Encode(w, args, local) if w.name == "encode" else Routed(w, args, local)
+    L = eng.L
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        eng.step()
+    torch.cuda.synchronize()
+    if args.profile_steps:
+        for _ in range(args.profile_steps):
+            eng.step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    planted_ok = None
+    if w.name != "encode":
+        bad = eng.check_planted()
+        planted_ok = bad == 0
+
+    # ---- timed region: K steps, inputs resident in HBM
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+           for _ in range(args.steps)]
+    for row in evs:
+        for a, b in row:
+            a.record()
+            b.record()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = msa.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_uuid(local)) as clk:
+        start.record()
+        for i in range(args.steps):
+            eng.step(evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+    barrier()
+    launches = (msa.launch_count() - launches0) / args.steps
+    ms = start.elapsed_time(stop) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = eng.units_per_step() * world / (ms / 1e3)
+    kern_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.steps) for l in range(L)]
+    kern_avg_ms = statistics.mean(kern_ms)
+
+    # ---- end to end through the public API: host inputs in, host results out
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(eng, w, args, world, unit)
+
+    peak, peak_kind = measured_peaks()
+    if w.name == "encode":
+        kbytes = eng.kernel_bytes_per_launch()
+        kname, ksrc = "encode_pool_kernel", "routed_sparse_attention_msa_b200/csrc/encode.cu"
+    else:
+        kbytes = eng.score_bytes_per_launch()
+        kname = "score_tc_kernel" if args.score_kernel in ("auto", "tc") else "score_simt_kernel"
+        ksrc = ("routed_sparse_attention_msa_b200/csrc/score_tc.cu" if kname == "score_tc_kernel"
+                else "routed_sparse_attention_msa_b200/csrc/score.cu")
+    achieved = kbytes / (kern_avg_ms / 1e3) / 1e9
+    traffic = traffic_for(kname, ksrc, w.name)
+    roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+            "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": kern_avg_ms * 1e3,
+            "launches_per_step": L}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        if w.name == "encode":
+            r = encode_cpu_baseline(w, n_docs=2)
+            cpu = {"value": r["tokens"] / r["seconds"], "unit": unit, "cores": 1, "kind": "oracle",
+                   "sample": f"2 documents x 4096 tokens, one layer: {r['seconds']:.1f} s"}
+        else:
+            dco, _ = w.index()
+            r = cpu_baseline(w, max_chunks=None if dco[-1] <= 2_000_000 else 2_000_000)
+            cpu = {"value": r["tokens"] / r["seconds"], "unit": unit, "cores": 1, "kind": "oracle",
+                   "sample": (f"one routing layer ({r['chunks']} chunks, {r['tokens']} memory tokens x sequences): "
+                              f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
+
+    extra = {"decode_latency_us_per_layer": 1e3 * ms / L}
+    if planted_ok is not None:
+        extra["planted_sets_retrieved"] = planted_ok
+    if w.name != "encode" and w.content_on_host:
+        extra["host_content_banks"] = eng.n_content
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, eng, args, extra), "parallelism": f"replicas{world}",
+            "e2e": e2e, "gpu_launches": launches, "roofline": roof, "cpu_baseline": cpu,
+            "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(eng, w, args, world, unit):
+    """Same metric through the C ABI, with the step's inputs copied from pinned
+    host buffers and its results read back inside the timed region."""
+    import torch
+    if w.name == "encode":
+        return None  # the offline encode's input is the resident corpus; no per-step host input
+    L = eng.L
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype).pin_memory()  # noqa: E731
+    h_qr = [pin(t) for t in eng.qr_d]
+    h_q = [pin(t) for t in eng.q_d]
+    for src, dst in ((eng.qr_d, h_qr), (eng.q_d, h_q)):
+        for s, d_ in zip(src, dst):
+            d_.copy_(s)
+    # the decoded token's new local K/V row (one per sequence): last local slot
+    last = eng.loc_off[1:] - 1
+    idx = torch.from_numpy(last.astype(np.int64)).cuda()
+    h_k = [pin(t[idx]) for t in eng.kl_d]
+    h_v = [pin(t[idx]) for t in eng.vl_d]
+    for l in range(L):
+        h_k[l].copy_(eng.kl_d[l][idx])
+        h_v[l].copy_(eng.vl_d[l][idx])
+    h_out = [pin(t) for t in eng.out]
+    h_ids = [pin(t) for t in eng.ids]
+    h2d = sum(t.numel() * t.element_size() for lst in (h_qr, h_q, h_k, h_v) for t in lst)
+    d2h = sum(t.numel() * t.element_size() for lst in (h_out, h_ids) for t in lst)
+
+    def step():
+        for l in range(L):
+            eng.qr_d[l].copy_(h_qr[l], non_blocking=True)
+            eng.q_d[l].copy_(h_q[l], non_blocking=True)
+            eng.kl_d[l][idx] = h_k[l].cuda(non_blocking=True)
+            eng.vl_d[l][idx] = h_v[l].cuda(non_blocking=True)
+        eng.step()
+        for l in range(L):
+            h_out[l].copy_(eng.out[l], non_blocking=True)
+            h_ids[l].copy_(eng.ids[l], non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(5, args.steps // 2)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": eng.units_per_step() * world / (ms / 1e3), "unit": unit, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -88,6 +88,12 @@ def normal_bf16_device(ptr: int, n: int, tensor_id: int, index0: int = 0, sigma:
         raise RuntimeError(f"synthetic fill kernel failed (cudaError {rc})")
 
 
+def normal_bf16_host_into(ptr: int, n: int, tensor_id: int, index0: int = 0, sigma: float = 1.0,
+                          seed: int = SEED) -> None:
+    """Like ``normal_bf16_host`` but writes into existing host memory at ``ptr``."""
+    _load().synth_normal_bf16_host(ctypes.c_void_p(ptr), int(n), seed, tensor_id, int(index0), float(sigma))
+
+
 def u64_host(n: int, tensor_id: int, index0: int = 0, seed: int = SEED) -> np.ndarray:
     out = np.empty(int(n), np.uint64)
     if n:
