@@ -173,6 +173,35 @@ msa_status msa_route(const msa_bank_layer* bank, const uint16_t* qr, const int32
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Route without a workspace. The pages have no counterpart: this is an
+ * interface addition of the library.
+ *
+ * For callers that cannot allocate device memory, such as a serving process
+ * whose framework reserves all of HBM for its own pool and forbids further
+ * cudaMalloc, or a latency-critical loop that cannot accept cudaMalloc's
+ * implicit device-wide synchronisation. msa_route_static computes exactly what
+ * msa_route computes, with the same arguments minus the workspace, and
+ * allocates nothing. Its scratch is one fixed array of
+ * MSA_ROUTE_STATIC_SCRATCH_BYTES in the library's device memory, which every
+ * GPU that loads the library holds until the process exits.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current). Make that first call before any
+ *    stream capture.
+ *  - A call whose scratch need (msa_route_workspace) exceeds the array
+ *    returns MSA_ERR_CAPACITY and enqueues nothing.
+ *  - All calls on a device share the one array; it keeps the last call's
+ *    contents, and every call first clears the part that must start at zero.
+ *    Calls that overlap on the GPU (different streams, or different threads
+ *    without ordering between them) race on the array and give wrong
+ *    results; order them on one stream.
+ * ---------------------------------------------------------------------- */
+#define MSA_ROUTE_STATIC_SCRATCH_BYTES ((size_t)4 << 20) /* 4 MiB */
+
+msa_status msa_route_static(const msa_bank_layer* bank, const uint16_t* qr, const int32_t* q_seq_off,
+                            int32_t n_seq, int32_t n_rows, int32_t top_k, float eps,
+                            int32_t* top_ids, float* top_scores, float* all_doc_scores, void* stream);
+
+/* ------------------------------------------------------------------------
  * Gather (context assembly).
  *
  * For each sequence s, the chunks of its selected documents top_ids[s, :] are

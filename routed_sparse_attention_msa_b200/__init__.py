@@ -88,13 +88,14 @@ _sig("msa_encode", [ctypes.POINTER(EncodeArgsC), P])
 _sig("msa_bank_norms", [P, i64, i32, i32, f32, P, P])
 _sig("msa_route_workspace", [ctypes.POINTER(BankLayerC), i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)])
 _sig("msa_route", [ctypes.POINTER(BankLayerC), P, P, i32, i32, i32, f32, P, P, P, P, ctypes.c_size_t, P])
+_sig("msa_route_static", [ctypes.POINTER(BankLayerC), P, P, i32, i32, i32, f32, P, P, P, P])
 _sig("msa_gather", [ctypes.POINTER(GatherArgsC), P])
 _sig("msa_attend_workspace", [ctypes.POINTER(AttendArgsC), ctypes.POINTER(ctypes.c_size_t)])
 _sig("msa_attend", [ctypes.POINTER(AttendArgsC), P, ctypes.c_size_t, P])
 _sig("msa_sync_check", [P])
 
 EXPORTS = ["msa_status_string", "msa_last_error", "msa_version", "msa_encode_plan", "msa_encode",
-           "msa_bank_norms", "msa_route_workspace", "msa_route", "msa_gather", "msa_attend_workspace",
+           "msa_bank_norms", "msa_route_workspace", "msa_route", "msa_route_static", "msa_gather", "msa_attend_workspace",
            "msa_attend", "msa_sync_check"]
 
 
@@ -222,6 +223,21 @@ def route(bank: BankLayer, qr, q_seq_off_host, top_k: int, top_ids, top_scores, 
     _check(_lib.msa_route(ctypes.byref(b), _ptr(qr), qso.ctypes.data, qso.size - 1, qr.shape[0], top_k, eps,
                           _ptr(top_ids), _ptr(top_scores), _ptr(all_doc_scores), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream)), "msa_route")
+
+
+ROUTE_STATIC_SCRATCH_BYTES = 4 << 20  # MSA_ROUTE_STATIC_SCRATCH_BYTES
+
+
+def route_static(bank: BankLayer, qr, q_seq_off_host, top_k: int, top_ids, top_scores, all_doc_scores=None,
+                 eps: float = 1e-8, stream=None) -> None:
+    """Route one layer without a workspace, for callers that may not allocate
+    device memory: the library's fixed device scratch is used instead. Same
+    results as ``route``. Calls on one device must not overlap on the GPU."""
+    b = bank.c()
+    qso = _host_i32(q_seq_off_host)
+    _check(_lib.msa_route_static(ctypes.byref(b), _ptr(qr), qso.ctypes.data, qso.size - 1, qr.shape[0], top_k, eps,
+                                 _ptr(top_ids), _ptr(top_scores), _ptr(all_doc_scores), _stream(stream)),
+           "msa_route_static")
 
 
 # ------------------------------------------------------------------ gather
