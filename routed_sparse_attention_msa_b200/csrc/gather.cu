@@ -60,8 +60,11 @@ __global__ void __launch_bounds__(1024) gather_index_kernel(
   }
 }
 
-// One warp per selected row: 2 x hkv x 256 B read from mapped host memory
-// with 16-byte loads, written to the staging buffers.
+// One warp per selected row: 2 x hkv x 256 B read from mapped host memory.
+// Every lane issues all of its 16-byte loads (K and V) before its first store
+// so that each warp keeps its whole row in flight over the host link.
+constexpr int kPullVecsPerLane = 4;  // hkv * 128 * 2 B / 16 B / 32 lanes, for hkv <= 8
+
 __global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint16_t* __restrict__ vbar,
                                    const int64_t* __restrict__ sel_total,
                                    const int64_t* __restrict__ sel_chunk, int64_t cap, int hkv,
@@ -77,11 +80,24 @@ __global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint
     const uint4* sv = reinterpret_cast<const uint4*>(vbar + (size_t)c * hkv * kHeadDim);
     uint4* dk = reinterpret_cast<uint4*>(stage_k + (size_t)j * hkv * kHeadDim);
     uint4* dv = reinterpret_cast<uint4*>(stage_v + (size_t)j * hkv * kHeadDim);
-    for (int i = lane; i < vecs; i += 32) {
-      uint4 a = sk[i];
-      uint4 b = sv[i];
-      dk[i] = a;
-      dv[i] = b;
+    for (int i0 = 0; i0 < vecs; i0 += 32 * kPullVecsPerLane) {
+      uint4 a[kPullVecsPerLane], b[kPullVecsPerLane];
+#pragma unroll
+      for (int u = 0; u < kPullVecsPerLane; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i < vecs) {
+          a[u] = sk[i];
+          b[u] = sv[i];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPullVecsPerLane; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i < vecs) {
+          dk[i] = a[u];
+          dv[i] = b[u];
+        }
+      }
     }
   }
 }

@@ -9,20 +9,25 @@
 // and all keys are distinct. A document that was never scored (no chunks)
 // has score word 0, below every real score.
 //
-// k <= 32: each warp keeps its best k keys sorted across lanes; a batch of 32
-// new keys is filtered against the k-th key with one ballot and the few
-// survivors are inserted by shuffles. CTAs take slices of the documents; the
-// last CTA of a sequence to finish (atomic ticket, no waiting) merges the
-// slices' candidates. k > 32: one CTA per sequence runs an 8-pass radix select
-// on the keys, collects the k keys at or above the k-th and sorts them.
+// k <= 16: each warp keeps its best 16 keys sorted across lanes 0..15. A batch
+// of 32 new keys is first tested against the 16th key with one ballot (after
+// the first batches almost every batch is skipped); otherwise the batch is
+// sorted by a 32-lane bitonic network and merged with the list by one
+// bitonic merge (the list in lanes 0..15, the batch's best 16 reversed into
+// lanes 16..31). Warps, then CTAs, are combined by the same merge. The last
+// CTA of a sequence to finish (atomic ticket, no waiting) merges the CTAs'
+// lists. 16 < k <= 32: the same structure with per-key insertion by shuffles.
+// k > 32: one CTA per sequence runs an 8-pass radix select on the keys,
+// collects the k keys at or above the k-th and sorts them.
 #include "msa_internal.cuh"
 
 namespace msa {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kDocsPerWarp = 512;
+constexpr int kDocsPerWarp = 128;
 constexpr int kDocsPerCta = kWarps * kDocsPerWarp;
+constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ uint64_t doc_key64(uint32_t score_key, int64_t doc) {
   return ((uint64_t)score_key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)doc);
@@ -47,6 +52,41 @@ __device__ __forceinline__ void warp_insert(uint64_t& list, uint64_t key, int k,
     m &= ~(1u << src);
     m &= __ballot_sync(0xffffffffu, key > thr);
   }
+}
+
+// 32 keys, one per lane, sorted descending across the warp.
+__device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t x, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t y = __shfl_xor_sync(kFull, x, stride);
+      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+      x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+    }
+  }
+  return x;
+}
+
+// list: lanes 0..15 hold 16 keys sorted descending. other: lanes 0..15 hold
+// another such list. Returns the best 16 of both, sorted, in lanes 0..15.
+__device__ __forceinline__ uint64_t warp_merge16(uint64_t list, uint64_t other, int lane) {
+  const uint64_t rev = __shfl_sync(kFull, other, 31 - lane);  // lane 16+i <- other[15-i]
+  uint64_t x = lane < 16 ? list : rev;                        // bitonic: descending then ascending
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t y = __shfl_xor_sync(kFull, x, stride);
+    x = (lane & stride) == 0 ? (x > y ? x : y) : (x < y ? x : y);
+  }
+  return x;
+}
+
+// Fold one batch of 32 keys (one per lane) into the list (lanes 0..15).
+__device__ __forceinline__ void warp_fold32(uint64_t& list, uint64_t key, int lane) {
+  const uint64_t thr = __shfl_sync(kFull, list, 15);
+  if (!__any_sync(kFull, key > thr)) return;
+  const uint64_t sorted = warp_sort32_desc(key, lane);
+  list = warp_merge16(list, sorted, lane);
 }
 
 __device__ __forceinline__ void write_result(uint64_t key, int32_t* ids, float* scores) {
@@ -102,6 +142,66 @@ __global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(
   }
   const int kk = k < n_docs ? k : (int)n_docs;
   if (lane < kk) write_result(fin, top_ids + (size_t)s * kk + lane, top_scores + (size_t)s * kk + lane);
+  if (lane == 0) tickets[s] = 0u;  // ready for the next call
+}
+
+__global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
+    const uint32_t* __restrict__ doc_key, int64_t n_docs, int k, uint64_t* __restrict__ cand,
+    unsigned* __restrict__ tickets, int32_t* __restrict__ top_ids, float* __restrict__ top_scores,
+    float* __restrict__ all_scores) {
+  __shared__ uint64_t s_lists[kWarps][16];
+  __shared__ bool s_last;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int s = blockIdx.y;
+  const int part = blockIdx.x;
+  const int n_parts = gridDim.x;
+  const uint32_t* keys = doc_key + (size_t)s * n_docs;
+
+  // keys of this warp's slice, all loads issued before any merging
+  const int64_t w0 = (int64_t)part * kDocsPerCta + (int64_t)wid * kDocsPerWarp;
+  constexpr int kIt = kDocsPerWarp / 32;
+  uint64_t kv[kIt];
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int64_t doc = w0 + it * 32 + lane;
+    kv[it] = 0;
+    if (doc < n_docs) {
+      const uint32_t sk = keys[doc];
+      kv[it] = doc_key64(sk, doc);
+      if (all_scores) all_scores[(size_t)s * n_docs + doc] = unord_f32(sk);
+    }
+  }
+  uint64_t list = warp_sort32_desc(kv[0], lane);
+#pragma unroll
+  for (int it = 1; it < kIt; ++it) warp_fold32(list, kv[it], lane);
+  if (lane < 16) s_lists[wid][lane] = list;
+  __syncthreads();
+  if (wid == 0) {
+    uint64_t merged = lane < 16 ? s_lists[0][lane] : 0ull;
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) merged = warp_merge16(merged, lane < 16 ? s_lists[w][lane] : 0ull, lane);
+    if (lane < 16) cand[((size_t)s * n_parts + part) * 16 + lane] = merged;
+    __threadfence();
+    unsigned t = 0;
+    if (lane == 0) t = atomicAdd(tickets + s, 1u);
+    t = __shfl_sync(kFull, t, 0);
+    s_last = (t == (unsigned)(n_parts - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // last CTA: every warp merges a share of the CTAs' lists, then warp 0 merges the warps'
+  const uint64_t* c = cand + (size_t)s * n_parts * 16;
+  uint64_t acc = 0;
+  for (int pp = wid; pp < n_parts; pp += kWarps)
+    acc = warp_merge16(acc, lane < 16 ? __ldcg(c + (size_t)pp * 16 + lane) : 0ull, lane);
+  if (lane < 16) s_lists[wid][lane] = acc;
+  __syncthreads();
+  if (wid != 0) return;
+  uint64_t fin = lane < 16 ? s_lists[0][lane] : 0ull;
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) fin = warp_merge16(fin, lane < 16 ? s_lists[w][lane] : 0ull, lane);
+  if (lane < k) write_result(fin, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
   if (lane == 0) tickets[s] = 0u;  // ready for the next call
 }
 
@@ -188,7 +288,8 @@ __global__ void __launch_bounds__(1024) topk_radix_kernel(
 size_t topk_workspace(int n_seq, int64_t n_docs, int k) {
   int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;
   if (k > 32) return 256;
-  return align_up((size_t)n_seq * parts * k * sizeof(uint64_t), 256) +
+  const int kc = k <= 16 ? 16 : k;
+  return align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256) +
          align_up((size_t)n_seq * sizeof(unsigned), 256);
 }
 
@@ -198,13 +299,19 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
   if (k > n_docs) k = (int)n_docs;
   if (k <= 32) {
     int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;
+    const int kc = k <= 16 ? 16 : k;
     uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
     unsigned* tickets = reinterpret_cast<unsigned*>(
-        reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * k * sizeof(uint64_t), 256));
+        reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256));
     dim3 grid((unsigned)parts, (unsigned)n_seq);
+    if (k <= 16) {
+      topk16_kernel<<<grid, kWarps * 32, 0, st>>>(doc_key, n_docs, k, cand, tickets, top_ids, top_scores,
+                                                  all_scores);
+      return launch_check("route: top-k (bitonic, k <= 16)");
+    }
     topk_warp_kernel<<<grid, kWarps * 32, 0, st>>>(doc_key, n_docs, k, cand, tickets, top_ids,
                                                    top_scores, all_scores);
-    return launch_check("route: top-k (warp)");
+    return launch_check("route: top-k (warp insertion)");
   }
   int pow2 = 1;
   while (pow2 < k) pow2 <<= 1;
