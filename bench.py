@@ -49,6 +49,9 @@ def parse_args():
                    help="host-tier content banks to allocate; layer l uses bank l mod this (0: one per layer "
                         "if host RAM allows)")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count (0: as defined)")
+    p.add_argument("--seqs", type=int, default=0, help="override the workload's sequence count (0: as defined)")
+    p.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
+                   help="replay each step as one CUDA graph (auto: on unless the copy-engine gather needs host syncs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile-steps", type=int, default=0,
@@ -145,6 +148,19 @@ def gpu_uuid(dev: int) -> str:
         return s if s.startswith("GPU-") else "GPU-" + s
     except Exception:
         return str(dev)
+
+
+def combine_ranks(ms: float, units_per_step: float, world: int, device="cuda"):
+    """Replicas: every rank times its own copy of the workload; the job's time
+    is the slowest rank's (max over ranks) and its throughput counts the units
+    of all ranks. Returns (value, ms)."""
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return units_per_step * world / (ms / 1e3), ms
 
 
 # --------------------------------------------------------- workload engine
@@ -339,11 +355,9 @@ class Encode:
     def step(self, evs=None):
         for l in range(self.L):
             if evs is not None:
-                evs[l][0].record()
+                self.msa.score_events(evs[l][0], evs[l][1])  # around the pooling kernel
             self.msa.encode(*self.inp, self.off_d, self.C, self.out, chunk=self.w.chunk,
                             rope_theta=self.w.rope_theta, eps=self.w.eps)
-            if evs is not None:
-                evs[l][1].record()
 
     def units_per_step(self):
         return float(self.w.memory_tokens) * self.L
@@ -479,6 +493,8 @@ def run_ours(args):
     import routed_sparse_attention_msa_b200 as msa
     msa.set_score_kernel(args.score_kernel)
     w = synth.workload(args.workload)
+    if args.seqs:
+        w.n_seq = args.seqs
     metric, unit = metric_of(w.name)
     eng = Encode(w, args, local) if w.name == "encode" else Routed(w, args, local)
     L = eng.L
@@ -504,8 +520,29 @@ def run_ours(args):
         planted_ok = bad == 0
 
     # ---- timed region: K steps, inputs resident in HBM
+    use_graph = args.graph == "on" or (args.graph == "auto" and not (
+        w.name != "encode" and w.content_on_host and args.gather == "copy"))
+    graph = None
+    if use_graph:
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+        for a_, b_ in gev:
+            a_.record()
+            b_.record()
+        torch.cuda.synchronize()
+        try:
+            graph = torch.cuda.CUDAGraph()
+            n0 = msa.launch_count()
+            with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+                eng.step(gev)
+            launches = msa.launch_count() - n0
+            graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture not possible here: fall back to eager launches
+            print(f"# CUDA graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            graph = None
+    eng.run_step = (graph.replay if graph is not None else eng.step)
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-           for _ in range(args.steps)]
+           for _ in range(args.steps if graph is None else 0)]
     for row in evs:
         for a, b in row:
             a.record()
@@ -518,18 +555,21 @@ def run_ours(args):
     with ClockSampler(gpu_uuid(local)) as clk:
         start.record()
         for i in range(args.steps):
-            eng.step(evs[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                eng.step(evs[i])
         stop.record()
         torch.cuda.synchronize()
     barrier()
-    launches = (msa.launch_count() - launches0) / args.steps
+    if graph is None:
+        launches = (msa.launch_count() - launches0) / args.steps
     ms = start.elapsed_time(stop) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = eng.units_per_step() * world / (ms / 1e3)
-    kern_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.steps) for l in range(L)]
+    value, ms = combine_ranks(ms, eng.units_per_step(), world)
+    if graph is not None:  # events recorded by the last replay of the timed region
+        kern_ms = [a.elapsed_time(b) for a, b in gev]
+    else:
+        kern_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.steps) for l in range(L)]
     kern_avg_ms = statistics.mean(kern_ms)
 
     # ---- end to end through the public API: host inputs in, host results out
@@ -566,7 +606,7 @@ def run_ours(args):
                    "sample": (f"one routing layer ({r['chunks']} chunks, {r['tokens']} memory tokens x sequences): "
                               f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
 
-    extra = {"decode_latency_us_per_layer": 1e3 * ms / L}
+    extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None}
     if planted_ok is not None:
         extra["planted_sets_retrieved"] = planted_ok
     if w.name != "encode" and w.content_on_host:
@@ -616,7 +656,7 @@ def run_e2e(eng, w, args, world, unit):
             eng.q_d[l].copy_(h_q[l], non_blocking=True)
             eng.kl_d[l][idx] = h_k[l].cuda(non_blocking=True)
             eng.vl_d[l][idx] = h_v[l].cuda(non_blocking=True)
-        eng.step()
+        eng.run_step()
         for l in range(L):
             h_out[l].copy_(eng.out[l], non_blocking=True)
             h_ids[l].copy_(eng.ids[l], non_blocking=True)
@@ -632,12 +672,8 @@ def run_e2e(eng, w, args, world, unit):
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": eng.units_per_step() * world / (ms / 1e3), "unit": unit, "h2d_bytes_per_step": h2d,
+    value, ms = combine_ranks(ms, eng.units_per_step(), world)
+    return {"value": value, "unit": unit, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 

@@ -271,8 +271,11 @@ msa_status launch_encode(const msa_encode_args& a, cudaStream_t st) {
   int heads = a.hkv > a.hr ? a.hkv : a.hr;
   int threads = 32 * ((heads + 1) / 2);  // whole warps: the norm reduction shuffles full warps
   int64_t grid = a.n_chunks < 148 * 40 ? a.n_chunks : 148 * 40;
+  record_debug_event(0, st);
   encode_pool_kernel<<<(unsigned)grid, threads, 0, st>>>(p);
-  return launch_check("encode: pooling");
+  msa_status s2 = launch_check("encode: pooling");
+  record_debug_event(1, st);
+  return s2;
 }
 
 msa_status launch_bank_norms(const uint16_t* kbar_r, int64_t n_chunks, int hr, float eps,

@@ -33,6 +33,18 @@ msa_status cuda_fail(cudaError_t e, const char* what) {
   return MSA_ERR_CUDA;
 }
 
+void record_debug_event(int which, cudaStream_t st) {
+  cudaEvent_t ev = g_score_ev[which];
+  if (!ev) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+  if (which == 1) g_score_ev[0] = g_score_ev[1] = nullptr;
+}
+
 msa_status launch_check(const char* what) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   cudaError_t e = cudaGetLastError();
@@ -112,9 +124,11 @@ int msa_debug_set_score_kernel(int which) {
 // goes through launch_check). Benchmark instrumentation.
 long long msa_debug_launch_count(void) { return g_launches.load(); }
 
-// The calling thread's next msa_route records `begin` and `end` (cudaEvent_t)
-// on its stream immediately around the scoring kernel, then forgets them.
-// Benchmark instrumentation: it times the scoring kernel inside a real step.
+// The calling thread's next msa_route (or msa_encode) records `begin` and
+// `end` (cudaEvent_t) on its stream immediately around its main kernel (the
+// scoring kernel, or the pooling kernel), then forgets them. Under stream
+// capture the records become external event nodes, so they fire on every
+// replay. Benchmark instrumentation: it times that kernel inside a real step.
 void msa_debug_score_events(void* begin, void* end) {
   g_score_ev[0] = (cudaEvent_t)begin;
   g_score_ev[1] = (cudaEvent_t)end;
@@ -217,10 +231,9 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   if (b->n_chunks > 0) {
     bool tc = g_score_kernel == 2 || (g_score_kernel == 0 && score_tc_supported(p));
     if (tc && !score_tc_supported(p)) return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
-    if (g_score_ev[0]) cudaEventRecord(g_score_ev[0], st);
+    record_debug_event(0, st);
     s = tc ? launch_score_tc(p, st) : launch_score_simt(p, st);
-    if (g_score_ev[1]) cudaEventRecord(g_score_ev[1], st);
-    g_score_ev[0] = g_score_ev[1] = nullptr;
+    record_debug_event(1, st);
     if (s != MSA_OK) return s;
   }
   int k = top_k < b->n_docs ? top_k : (int)b->n_docs;

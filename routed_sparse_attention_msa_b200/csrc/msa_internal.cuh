@@ -13,6 +13,8 @@ namespace msa {
 msa_status fail(msa_status s, const char* fmt, ...);
 msa_status cuda_fail(cudaError_t e, const char* what);
 msa_status launch_check(const char* what);
+// Benchmark instrumentation: records the pending debug event `which` (0 begin, 1 end) on st.
+void record_debug_event(int which, cudaStream_t st);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

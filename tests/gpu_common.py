@@ -56,10 +56,10 @@ class DevBank:
         self.kbar = self.vbar = None
         if content:
             if on_host:
-                self.kbar = torch.from_numpy(host_normal((self.C, hkv, 128), synth.tid("kbar", layer)).view(
-                    np.int16)).view(torch.bfloat16).pin_memory()
-                self.vbar = torch.from_numpy(host_normal((self.C, hkv, 128), synth.tid("vbar", layer)).view(
-                    np.int16)).view(torch.bfloat16).pin_memory()
+                self.kbar = torch.empty((self.C, hkv, 128), dtype=torch.bfloat16, pin_memory=True)
+                self.vbar = torch.empty((self.C, hkv, 128), dtype=torch.bfloat16, pin_memory=True)
+                synth.normal_bf16_host_into(self.kbar.data_ptr(), self.kbar.numel(), synth.tid("kbar", layer))
+                synth.normal_bf16_host_into(self.vbar.data_ptr(), self.vbar.numel(), synth.tid("vbar", layer))
             else:
                 self.kbar = dev_normal((self.C, hkv, 128), synth.tid("kbar", layer))
                 self.vbar = dev_normal((self.C, hkv, 128), synth.tid("vbar", layer))

@@ -1,0 +1,233 @@
+"""GPU parity at the five workloads' full sizes, in the launch configuration
+bench.py times, against the CPU oracle.
+
+Where the oracle finishes in seconds it runs in full (1M-token decode on every
+layer, 1M-token prefill on one layer, one whole 100M-token layer); elsewhere it
+scores sampled documents one by one (a sub-bank holding only those documents'
+chunks gives exactly their scores), and the property that holds at any size
+is checked: every sequence's routed set is its planted set and every
+unselected document scores below the k-th selected one.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.gpu_common import DevBank, bits, check_topk, from_bits, gap_at_k, host_normal, route_gpu
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def msa():
+    import routed_sparse_attention_msa_b200 as m
+    return m
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def sub_bank(bank: DevBank, docs):
+    """Pooled routing keys of the given documents only, regenerated on the host."""
+    parts, nch = [], []
+    for d in docs:
+        c0, c1 = int(bank.dco[d]), int(bank.dco[d + 1])
+        parts.append(host_normal((c1 - c0, bank.hr, 128), synth.tid("kbar_r", bank.layer), index0=c0 * bank.hr * 128))
+        nch.append(c1 - c0)
+    kr = np.concatenate(parts) if parts else np.zeros((0, bank.hr, 128), np.uint16)
+    return kr, np.concatenate([[0], np.cumsum(nch)]).astype(np.int64)
+
+
+def check_sampled(bank, qr, qso, ids, sc, alls, plans, n_random=100, seed=0):
+    """Oracle scores of the planted documents and of random others, per sequence,
+    against the GPU's; planted sets retrieved; top-k property on the GPU scores."""
+    rng = np.random.default_rng(seed)
+    S, k = ids.shape
+    for s in range(S):
+        planted = list(plans.docs[s])
+        others = [int(d) for d in rng.choice(bank.n_docs, n_random, replace=False) if d not in planted]
+        docs = planted + others
+        kr, dco = sub_bank(bank, docs)
+        rows = slice(int(qso[s]), int(qso[s + 1]))
+        _, _, o_all = oracle.route(kr, dco, np.ascontiguousarray(qr[rows]), [0, rows.stop - rows.start], 1)
+        g = alls[s][docs]
+        finite = np.isfinite(o_all[0])
+        np.testing.assert_allclose(g[finite], o_all[0][finite], atol=1e-3, rtol=0)
+        assert set(ids[s].tolist()) == set(planted), s
+        # top-k property over every document, on the GPU's own scores
+        unselected = np.delete(alls[s], ids[s])
+        assert unselected.max() < sc[s].min()
+
+
+# ------------------------------------------------------------------ tiny
+
+def test_tiny_full(msa):
+    w = synth.workload("tiny")
+    bank = DevBank(w.doc_tok_off, 0, content=True)
+    qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [w.route_rows], w.top_k,
+                                               w.n_needles, w.hr, w.d, 0)
+    ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
+    o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, w.top_k)
+    assert gap_at_k(o_all[0], w.top_k) >= 1e-2
+    np.testing.assert_array_equal(ids, o_ids)
+    np.testing.assert_allclose(alls, o_all, atol=1e-3, rtol=0)
+
+
+# -------------------------------------------------------------------- 1m
+
+def test_1m_decode_all_layers_and_prefill(msa):
+    w = synth.workload("1m")
+    n_exact = 0
+    for layer in range(w.n_layers):
+        bank = DevBank(w.doc_tok_off, layer, content=False)
+        qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1], w.top_k, w.n_needles,
+                                                   w.hr, w.d, layer)
+        ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
+        o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, w.top_k)
+        n_exact += check_topk(ids, sc, o_ids, o_sc, o_all)
+        np.testing.assert_allclose(alls, o_all, atol=1e-3, rtol=0)
+        if layer == 0:
+            # 128-row prefill of the same layer, full oracle
+            qp, qsp, planp = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [w.prefill_rows],
+                                                        w.top_k, w.n_needles, w.hr, w.d, layer, call=1)
+            pid, psc, pall = route_gpu(bank, qp, qsp, w.top_k)
+            o_pid, o_psc, o_pall = oracle.route(bank.host_kbar_r(), bank.dco, qp, qsp, w.top_k)
+            assert check_topk(pid, psc, o_pid, o_psc, o_pall) == 1
+            np.testing.assert_allclose(pall, o_pall, atol=1e-3, rtol=0)
+            assert set(pid[0].tolist()) == set(planp.docs[0])
+        del bank
+    assert n_exact >= w.n_layers - 1  # rank-k gap >= 1e-2 on (almost) every layer
+
+
+# ------------------------------------------------------------------- 10m
+
+def test_10m_prefill_and_decode_sampled(msa):
+    w = synth.workload("10m")
+    bank = DevBank(w.doc_tok_off, 0, content=True)
+    # prefill: 16 sequences x 64 rows
+    qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [w.prefill_rows] * w.n_seq,
+                                               w.top_k, w.n_needles, w.hr, w.d, 0, call=1)
+    ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
+    check_sampled(bank, qr, qso, ids, sc, alls, plan, n_random=40)
+    # decode: one row per sequence; sequence 0 against the full oracle
+    qd, qsd, pland = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1] * w.n_seq, w.top_k,
+                                                w.n_needles, w.hr, w.d, 0)
+    ids, sc, alls = route_gpu(bank, qd, qsd, w.top_k)
+    check_sampled(bank, qd, qsd, ids, sc, alls, pland, n_random=100)
+    o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, np.ascontiguousarray(qd[:1]), [0, 1], w.top_k)
+    check_topk(ids[:1], sc[:1], o_ids, o_sc, o_all)
+    np.testing.assert_allclose(alls[0], o_all[0], atol=1e-3, rtol=0)
+    # gather + attend of the decode step (16 rows, 65 local keys each) against the oracle chain
+    S, L = w.n_seq, w.loc_len
+    top_d = torch.from_numpy(ids).cuda()
+    cap = S * w.top_k * bank.layer_c.max_doc_chunks
+    sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    sel = torch.empty(cap, dtype=torch.int64, device="cuda")
+    msa.gather(bank.layer_c, top_d, w.top_k, sel_off, sel)
+    o_off, o_sel = oracle.gather(ids, bank.dco)
+    np.testing.assert_array_equal(sel_off.cpu().numpy(), o_off)
+    q = host_normal((S, w.hq, 128), synth.tid("q_att", 0))
+    kl = host_normal((S * L, w.hkv, 128), synth.tid("k_loc", 0))
+    vl = host_normal((S * L, w.hkv, 128), synth.tid("v_loc", 0))
+    qso_a, qst, lo = np.arange(S + 1), np.full(S, L - 1), np.arange(S + 1) * L
+    out = torch.empty((S, w.hq, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((S, w.hq, 128), dtype=torch.float32, device="cuda")
+    args = (from_bits(q), qso_a, qst, from_bits(kl), from_bits(vl), lo, bank.kbar, bank.vbar, sel_off, sel, cap)
+    ws = torch.empty(msa.attend_workspace(*args), dtype=torch.uint8, device="cuda")
+    msa.attend(*args, out, ws, out_f32=of, pos_offset=float(w.top_k))
+    msa.sync_check()
+    kh, vh = bank.host_content()
+    o_out, _ = oracle.attend(q, qso_a, qst, kl, vl, lo, kh, vh, o_off, o_sel, pos_offset=float(w.top_k))
+    assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+
+
+# ------------------------------------------------------------------ 100m
+
+def test_100m_layer_full_oracle_host_tier(msa):
+    """One whole 100M-token layer (1,562,500 chunks) against the full oracle;
+    content in pinned host memory, device-pull gather, decode attention."""
+    w = synth.workload("100m")
+    bank = DevBank(w.doc_tok_off, 0, content=True, on_host=True)
+    qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1], w.top_k, w.n_needles,
+                                               w.hr, w.d, 0)
+    ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
+    kr_h = bank.host_kbar_r()
+    o_ids, o_sc, o_all = oracle.route(kr_h, bank.dco, qr, qso, w.top_k)
+    del kr_h
+    check_topk(ids, sc, o_ids, o_sc, o_all)
+    np.testing.assert_allclose(alls, o_all, atol=1e-3, rtol=0)
+    if gap_at_k(o_all[0], w.top_k) >= 1e-2:
+        assert set(ids[0].tolist()) == set(plan.docs[0])
+    # gather from pinned host memory + attend, against the oracle chain
+    cap = w.top_k * bank.layer_c.max_doc_chunks
+    top_d = torch.from_numpy(ids).cuda()
+    sel_off = torch.empty(2, dtype=torch.int64, device="cuda")
+    sel = torch.empty(cap, dtype=torch.int64, device="cuda")
+    sk = torch.empty((cap, w.hkv, 128), dtype=torch.bfloat16, device="cuda")
+    sv = torch.empty((cap, w.hkv, 128), dtype=torch.bfloat16, device="cuda")
+    msa.gather(bank.layer_c, top_d, w.top_k, sel_off, sel, sk, sv, mode=msa.GATHER_DEVICE_PULL)
+    o_off, o_sel = oracle.gather(ids, bank.dco)
+    L = w.loc_len
+    q = host_normal((1, w.hq, 128), synth.tid("q_att", 0))
+    kl = host_normal((L, w.hkv, 128), synth.tid("k_loc", 0))
+    vl = host_normal((L, w.hkv, 128), synth.tid("v_loc", 0))
+    out = torch.empty((1, w.hq, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((1, w.hq, 128), dtype=torch.float32, device="cuda")
+    args = (from_bits(q), [0, 1], [L - 1], from_bits(kl), from_bits(vl), [0, L], sk, sv, sel_off, None, cap)
+    ws = torch.empty(msa.attend_workspace(*args), dtype=torch.uint8, device="cuda")
+    msa.attend(*args, out, ws, out_f32=of, pos_offset=float(w.top_k))
+    msa.sync_check()
+    n = int(o_off[-1])
+    np.testing.assert_array_equal(bits(sk)[:n], bits(bank.kbar)[o_sel])
+    kh = bits(bank.kbar)[o_sel]
+    vh = bits(bank.vbar)[o_sel]
+    o_out, _ = oracle.attend(q, [0, 1], [L - 1], kl, vl, [0, L], kh, vh, o_off, np.arange(n, dtype=np.int64),
+                             pos_offset=float(w.top_k))
+    assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+
+
+# ---------------------------------------------------------------- encode
+
+def test_encode_10m_sampled_documents(msa):
+    w = synth.workload("encode")
+    n = w.memory_tokens
+    st = torch.cuda.current_stream().cuda_stream
+    inp = []
+    for kind, heads in (("k_tok", w.hkv), ("v_tok", w.hkv), ("kr_tok", w.hr)):
+        t = torch.empty((n, heads, w.d), dtype=torch.bfloat16, device="cuda")
+        synth.normal_bf16_device(t.data_ptr(), t.numel(), synth.tid(kind, 0), stream=st)
+        inp.append(t)
+    C, dco_h, _ = msa.encode_plan(w.doc_tok_off, w.chunk)
+    out = dict(kbar=torch.empty((C, w.hkv, w.d), dtype=torch.bfloat16, device="cuda"),
+               vbar=torch.empty((C, w.hkv, w.d), dtype=torch.bfloat16, device="cuda"),
+               kbar_r=torch.empty((C, w.hr, w.d), dtype=torch.bfloat16, device="cuda"),
+               kr_inv_norm=torch.empty((C, w.hr), dtype=torch.float32, device="cuda"),
+               doc_chunk_off=torch.empty(w.n_docs + 1, dtype=torch.int64, device="cuda"),
+               chunk_doc=torch.empty(C, dtype=torch.int32, device="cuda"))
+    msa.encode(*inp, torch.from_numpy(w.doc_tok_off).cuda(), C, out, rope_theta=w.rope_theta)
+    msa.sync_check()
+    del inp
+    np.testing.assert_array_equal(out["doc_chunk_off"].cpu().numpy(), dco_h)
+    for doc in [0, 1, 1234, w.n_docs - 1]:  # the last document has 1,664 tokens (26 chunks)
+        t0, t1 = int(w.doc_tok_off[doc]), int(w.doc_tok_off[doc + 1])
+        L = t1 - t0
+        ref = oracle.encode(host_normal((L, w.hkv, w.d), synth.tid("k_tok", 0), index0=t0 * w.hkv * w.d),
+                            host_normal((L, w.hkv, w.d), synth.tid("v_tok", 0), index0=t0 * w.hkv * w.d),
+                            host_normal((L, w.hr, w.d), synth.tid("kr_tok", 0), index0=t0 * w.hr * w.d),
+                            np.array([0, L], np.int64), rope_theta=w.rope_theta)
+        c0, c1 = int(dco_h[doc]), int(dco_h[doc + 1])
+        assert c1 - c0 == math.ceil(L / 64)
+        assert np.all(out["chunk_doc"][c0:c1].cpu().numpy() == doc)
+        for name in ["kbar", "vbar", "kbar_r"]:
+            g = oracle.bf16_to_f64(bits(out[name][c0:c1]))
+            o = oracle.bf16_to_f64(ref[name])
+            ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(o), 2.0 ** -126))) - 7)
+            assert np.all(np.abs(g - o) <= ulp + 2e-5), (doc, name)
+        np.testing.assert_allclose(out["kr_inv_norm"][c0:c1].cpu().numpy(), ref["kr_inv_norm"], rtol=2e-4)
