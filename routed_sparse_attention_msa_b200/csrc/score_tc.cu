@@ -180,7 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_invq = reinterpret_cast<float*>(tmem_slot + 4);  // [NB][8]
+  // per row block: query scales [NB][8], and for each column its sequence
+  // (-1 past the last row) and whether a sequence's run ends there
+  float* s_invq = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
+  int* s_seq = reinterpret_cast<int*>(s_invq + NB * kHeads);
+  int* s_end = s_seq + NB;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -283,6 +287,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row = 32 * q + lane;           // chunk within the tile
     const int et = threadIdx.x - 32 * kEpiWarp0;  // 0..127
+    auto load_block = [&](int t0) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int i = et; i < NB * kHeads; i += 128) {
+        const int t = t0 + i / kHeads;
+        s_invq[i] = t < a.n_rows ? a.invq[(size_t)t * kHeads + (i % kHeads)] : 0.f;
+      }
+      for (int i = et; i < NB; i += 128) {
+        const int t = t0 + i;
+        int sq = -1, end = 0;
+        if (t < a.n_rows) {
+          sq = seq_of_row(a.q_seq_off, a.n_seq, t);
+          end = (t + 1 == a.q_seq_off[sq + 1]) || (i == NB - 1) || (t + 1 == a.n_rows);
+        }
+        s_seq[i] = sq;
+        s_end[i] = end;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    };
+    if (a.n_nb == 1) load_block(0);
     int blk = 0;
     for (int tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
       const int64_t c = (int64_t)tile * kTileM + row;
@@ -307,55 +330,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane + o < 32 && dn == doc) same |= 1u << i;
       }
       const int doc_up = __shfl_up_sync(0xffffffffu, doc, 1);
-      const bool head = doc >= 0 && (lane == 0 || doc_up != doc);  // first lane of a document segment
+      const bool head = valid && (lane == 0 || doc_up != doc);  // first lane of a document segment
 
       bool ok = true;
       for (int nb = 0; nb < a.n_nb; ++nb, ++blk) {
         const int b = blk & 1;
-        const int t0 = nb * NB;
-        // this block's query scales, shared by the 128 epilogue threads
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        for (int i = et; i < NB * kHeads; i += 128) {
-          const int t = t0 + i / kHeads;
-          s_invq[i] = t < a.n_rows ? a.invq[(size_t)t * kHeads + (i % kHeads)] : 0.f;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (a.n_nb > 1) load_block(nb * NB);
         if (!mbar_wait(smem_u32(&tfull[b]), (blk >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float sacc[NB];
+        // Stream over the block's columns: the score of (row, column), a
+        // running max over the current sequence's columns, and a flush (warp
+        // max over the document's chunks, one atomic per document) wherever a
+        // sequence's run ends. Column metadata is uniform across the warp.
+        float m = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < NB; ++j) sacc[j] = 0.f;
+        for (int jh = 0; jh < NB; jh += 16) {
+          float v[kHeads][16];
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          float v[NB];
-          const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((b * kHeads + h) * NB);
-#pragma unroll
-          for (int j0 = 0; j0 < NB; j0 += 16) tmem_ld16(taddr + j0, v + j0);
+          for (int h = 0; h < kHeads; ++h)
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((b * kHeads + h) * NB + jh), v[h]);
           tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < NB; ++j) sacc[j] += v[j] * (invk[h] * s_invq[j * kHeads + h]);
-        }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&tempty[b]));
-
-        // max over each sequence's rows in this block, then over the
-        // document's chunks in this warp, then one atomic per document.
-        const int t_last = min(t0 + NB, a.n_rows) - 1;
-        const int s_first = seq_of_row(a.q_seq_off, a.n_seq, t0);
-        const int s_last = seq_of_row(a.q_seq_off, a.n_seq, t_last);
-        for (int sq = s_first; sq <= s_last; ++sq) {
-          const int jb = max(a.q_seq_off[sq], t0) - t0;
-          const int je = min(a.q_seq_off[sq + 1], t0 + NB) - t0;
-          float m = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < NB; ++j)
-            if (j >= jb && j < je) m = fmaxf(m, sacc[j]);
-#pragma unroll
-          for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
-            float mo = __shfl_down_sync(0xffffffffu, m, o);
-            if (same & (1u << i)) m = fmaxf(m, mo);
+          if (jh + 16 >= NB) {  // every accumulator of this buffer is in registers
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[b]));
           }
-          if (head && valid) atomicMax(a.doc_key + (size_t)sq * a.n_docs + doc, ord_f32(m));
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int jj = jh + j;
+            const int sq = s_seq[jj];
+            if (sq < 0) break;
+            const float4 qa = *reinterpret_cast<const float4*>(s_invq + jj * kHeads);
+            const float4 qb = *reinterpret_cast<const float4*>(s_invq + jj * kHeads + 4);
+            float sc = v[0][j] * (invk[0] * qa.x);
+            sc += v[1][j] * (invk[1] * qa.y);
+            sc += v[2][j] * (invk[2] * qa.z);
+            sc += v[3][j] * (invk[3] * qa.w);
+            sc += v[4][j] * (invk[4] * qb.x);
+            sc += v[5][j] * (invk[5] * qb.y);
+            sc += v[6][j] * (invk[6] * qb.z);
+            sc += v[7][j] * (invk[7] * qb.w);
+            m = fmaxf(m, sc);
+            if (s_end[jj]) {
+#pragma unroll
+              for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
+                const float mo = __shfl_down_sync(0xffffffffu, m, o);
+                if (same & (1u << i)) m = fmaxf(m, mo);
+              }
+              if (head) atomicMax(a.doc_key + (size_t)sq * a.n_docs + doc, ord_f32(m));
+              m = -INFINITY;
+            }
+          }
         }
       }
       if (!ok) break;
