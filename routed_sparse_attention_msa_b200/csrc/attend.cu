@@ -9,11 +9,14 @@
 //
 // Two kernels:
 //  1. rope_rows: rotates the query rows and the local keys once per call into
-//     fp32 copies (angles in double, so positions of any size keep full
-//     accuracy), and clears the merge tickets.
+//     fp32 copies, and clears the merge tickets. Each angle is formed and
+//     reduced modulo 2*pi in double, so positions of any size keep full
+//     accuracy, and then evaluated with sincosf.
 //  2. attend_split: split-K flash decoding. A CTA owns one kv head, a tile of
-//     query rows of one sequence (the GQA group's q heads x rows = 16 query
-//     vectors) and one contiguous slice of the key list. It walks the slice in
+//     query rows of one sequence (the GQA group's q heads x rows = 4, 8 or 16
+//     query vectors, the fewest that hold the sequence's rows: 4 for a decoding
+//     step with 4 q heads per kv head) and one contiguous slice of the key
+//     list. It walks the slice in
 //     blocks of 64 keys: the block's key and value rows are staged into
 //     shared memory with every load issued at once (decoding is bound by
 //     memory latency, a few hundred keys per head), then logits, an online
@@ -28,7 +31,7 @@
 namespace msa {
 namespace {
 
-constexpr int kVec = 16;       // query vectors per CTA (group x rows)
+constexpr int kMaxVec = 16;    // query vectors per CTA (group x rows): 4, 8 or 16
 constexpr int kKeyBlock = 64;  // keys per block
 constexpr int kThreads = 128;
 constexpr int kPad = 132;      // fp32 row stride in shared memory (bank-conflict free)
@@ -58,13 +61,14 @@ struct AttnParams {
   int32_t tile_off[kMaxSeq + 1];
 };
 
+template <int VEC>
 struct Smem {
-  float q[kVec][kHeadDim];
+  float q[VEC][kHeadDim];
   float k[kKeyBlock][kPad];
   float v[kKeyBlock][kPad];
-  float p[kVec][kKeyBlock];
-  float m[kVec], l[kVec], corr[kVec];
-  int g[kVec];
+  float p[VEC][kKeyBlock];
+  float m[VEC], l[VEC], corr[VEC];
+  int g[VEC];
   bool last;
 };
 
@@ -101,16 +105,25 @@ __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
   const uint16_t* src = (is_q ? p.q : p.k_loc) + rh * kHeadDim;
   float* dst = (is_q ? p.qrot : p.krot) + rh * kHeadDim;
   const double w = exp2(-2.0 * (double)i / (double)kHeadDim * p.log2_theta);
-  double sn, cs;
-  sincos(pos * w, &sn, &cs);
-  const double x0 = bf1(src[i]), x1 = bf1(src[i + 64]);
-  dst[i] = (float)(x0 * cs - x1 * sn);
-  dst[i + 64] = (float)(x0 * sn + x1 * cs);
+  const double ang = pos * w;
+  const double two_pi = 6.283185307179586476925286766559;
+  const float r = (float)(ang - two_pi * rint(ang / two_pi));  // in [-pi, pi]
+  float sn, cs;
+  sincosf(r, &sn, &cs);
+  const float x0 = bf1(src[i]), x1 = bf1(src[i + 64]);
+  dst[i] = x0 * cs - x1 * sn;
+  dst[i + 64] = x0 * sn + x1 * cs;
 }
 
+// VEC query vectors per CTA: logits give each key two threads of VEC/2
+// vectors; the softmax gives each warp VEC/4 vectors; P.V gives each thread 4
+// dimensions of VEC/4 vectors.
+template <int VEC>
 __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_constant__ AttnParams p) {
+  constexpr int VH = VEC / 2;  // vectors per thread in the logits
+  constexpr int VW = VEC / 4;  // vectors per warp (softmax) and per thread (P.V)
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  Smem<VEC>& S = *reinterpret_cast<Smem<VEC>*>(smem_raw);
 
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int sp_idx = blockIdx.x;
@@ -132,7 +145,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
   const size_t row_stride = (size_t)p.hkv * kHeadDim;
 
   // query vectors v = rr * group + gg
-  for (int idx = tid; idx < kVec * kHeadDim / 4; idx += kThreads) {
+  for (int idx = tid; idx < VEC * kHeadDim / 4; idx += kThreads) {
     const int v = idx / (kHeadDim / 4), e4 = idx % (kHeadDim / 4);
     const int rr = v / p.group, gg = v % p.group;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -140,16 +153,16 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
       x = reinterpret_cast<const float4*>(p.qrot + ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim)[e4];
     reinterpret_cast<float4*>(S.q[v])[e4] = x;
   }
-  if (tid < kVec) {
+  if (tid < VEC) {
     S.m[tid] = -INFINITY;
     S.l[tid] = 0.f;
     const int rr = tid / p.group;
     S.g[tid] = rr < nr ? g0 + rr : -1;  // -1: padding vector, sees nothing
   }
 
-  float acc[4][4];
+  float acc[VW][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < VW; ++i)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
   const int d0 = 4 * lane;
@@ -208,18 +221,18 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
       }
     }
     __syncthreads();
-    // ---- logits: thread -> one key, 8 query vectors
+    // ---- logits: thread -> one key, VH query vectors
     {
       const int jj = tid & (kKeyBlock - 1);
-      const int vh = (tid >> 6) * 8;
-      float dot[8];
+      const int vh = (tid >> 6) * VH;
+      float dot[VH];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) dot[v] = 0.f;
+      for (int v = 0; v < VH; ++v) dot[v] = 0.f;
 #pragma unroll 8
       for (int c = 0; c < kHeadDim / 4; ++c) {
         const float4 x = *reinterpret_cast<const float4*>(&S.k[jj][4 * c]);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < VH; ++v) {
           const float4 qa = *reinterpret_cast<const float4*>(&S.q[vh + v][4 * c]);
           dot[v] += x.x * qa.x + x.y * qa.y + x.z * qa.z + x.w * qa.w;
         }
@@ -227,17 +240,17 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
       const int64_t key = kb + jj;
       const int lj = key < n_mem ? -1 : (int)(key - n_mem);  // local key index, or -1
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
+      for (int v = 0; v < VH; ++v) {
         const int g = S.g[vh + v];
         const bool vis = jj < nb && g >= 0 && (lj < 0 || lj <= g);
         S.p[vh + v][jj] = vis ? dot[v] * p.scale : -INFINITY;
       }
     }
     __syncthreads();
-    // ---- online softmax: warp w owns vectors 4w .. 4w+3
+    // ---- online softmax: warp w owns vectors VW*w .. VW*w + VW-1
 #pragma unroll
-    for (int vi = 0; vi < 4; ++vi) {
-      const int v = 4 * wid + vi;
+    for (int vi = 0; vi < VW; ++vi) {
+      const int v = VW * wid + vi;
       const float x0 = S.p[v][lane], x1 = S.p[v][lane + 32];
       float bm = fmaxf(x0, x1);
 #pragma unroll
@@ -265,7 +278,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
     __syncthreads();
     // ---- P V: thread -> dims 4*lane .. +3 of vectors wid + 4i
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < VW; ++i) {
       const float corr = S.corr[wid + 4 * i];
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][e] *= corr;
@@ -273,7 +286,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
     for (int j = 0; j < nb; ++j) {
       const float4 x = *reinterpret_cast<const float4*>(&S.v[j][d0]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < VW; ++i) {
         const float pr = S.p[wid + 4 * i][j];
         acc[i][0] += pr * x.x;
         acc[i][1] += pr * x.y;
@@ -287,7 +300,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
   // ---- write: final rows, or a partial for the merge
   if (p.n_splits == 1) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < VW; ++i) {
       const int v = wid + 4 * i;
       const int rr = v / p.group, gg = v % p.group;
       if (rr >= nr) continue;
@@ -303,7 +316,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
     return;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < VW; ++i) {
     const int v = wid + 4 * i;
     const int rr = v / p.group, gg = v % p.group;
     if (rr >= nr) continue;
@@ -322,7 +335,7 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
   __threadfence();
   // ---- merge the splits of this (tile, kv head)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < VW; ++i) {
     const int v = wid + 4 * i;
     const int rr = v / p.group, gg = v % p.group;
     if (rr >= nr) continue;
@@ -355,13 +368,22 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
 }
 
 struct Shape {
-  int rt, n_tiles, n_splits, n_loc;
+  int vec, rt, n_tiles, n_splits, n_loc;
 };
 
 Shape plan(const msa_attend_args& a) {
   Shape sh;
   const int group = a.hq / a.hkv;
-  sh.rt = kVec / group;
+  int max_rows = 1;
+  for (int s = 0; s < a.n_seq; ++s) {
+    const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
+    max_rows = rows > max_rows ? rows : max_rows;
+  }
+  // query vectors per CTA: the GQA group times enough rows, 4 to 16
+  sh.vec = 4;
+  while (sh.vec < kMaxVec && sh.vec < group * max_rows) sh.vec *= 2;
+  if (sh.vec < group) sh.vec = group;
+  sh.rt = sh.vec / group;
   sh.n_tiles = 0;
   int max_loc = 0;
   for (int s = 0; s < a.n_seq; ++s) {
@@ -396,6 +418,19 @@ Layout layout(const msa_attend_args& a, const Shape& sh) {
   L.tickets = L.part_ml + align_up(np * 8, 256);
   L.total = L.tickets + align_up((size_t)sh.n_tiles * a.hkv * 4 + 4, 256);
   return L;
+}
+
+template <int VEC>
+msa_status launch_vec(const AttnParams& P, dim3 grid, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attend_split_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(Smem<VEC>));
+    if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
+    attr = true;
+  }
+  attend_split_kernel<VEC><<<grid, kThreads, sizeof(Smem<VEC>), st>>>(P);
+  return launch_check("attend: split-K with merge");
 }
 
 }  // namespace
@@ -442,16 +477,12 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   rope_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(P);
   msa_status s = launch_check("attend: rotate queries and local keys");
   if (s != MSA_OK) return s;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(Smem));
-    if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
-    attr = true;
-  }
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
-  attend_split_kernel<<<grid, kThreads, sizeof(Smem), st>>>(P);
-  return launch_check("attend: split-K with merge");
+  switch (sh.vec) {
+    case 4: return launch_vec<4>(P, grid, st);
+    case 8: return launch_vec<8>(P, grid, st);
+    default: return launch_vec<16>(P, grid, st);
+  }
 }
 
 }  // namespace msa
