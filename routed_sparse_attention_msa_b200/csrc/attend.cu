@@ -83,6 +83,8 @@ __device__ __forceinline__ int seq_of(const int32_t* off, int n_seq, int x) {
 
 // One thread per (row, head, pair) of the query rows, then of the local keys.
 __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < (int64_t)p.n_tiles * p.hkv) p.tickets[idx] = 0u;
   const int64_t nq = (int64_t)p.n_q * p.hq * 64;
@@ -124,6 +126,8 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
   constexpr int VW = VEC / 4;  // vectors per warp (softmax) and per thread (P.V)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem<VEC>& S = *reinterpret_cast<Smem<VEC>*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
 
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int sp_idx = blockIdx.x;
@@ -429,7 +433,8 @@ msa_status launch_vec(const AttnParams& P, dim3 grid, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
     attr = true;
   }
-  attend_split_kernel<VEC><<<grid, kThreads, sizeof(Smem<VEC>), st>>>(P);
+  cudaError_t e = launch_pdl(attend_split_kernel<VEC>, grid, dim3(kThreads), sizeof(Smem<VEC>), st, P);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: split-K with merge");
   return launch_check("attend: split-K with merge");
 }
 
@@ -474,7 +479,8 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   int64_t n = (int64_t)a.n_q * a.hq * 64 + (int64_t)sh.n_loc * a.hkv * 64;
   const int64_t nt = (int64_t)sh.n_tiles * a.hkv;
   if (n < nt) n = nt;
-  rope_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(P);
+  cudaError_t e = launch_pdl(rope_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, P);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: rotate queries and local keys");
   msa_status s = launch_check("attend: rotate queries and local keys");
   if (s != MSA_OK) return s;
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);

@@ -28,6 +28,8 @@ __global__ void doc_chunk_scan_kernel(const int64_t* __restrict__ doc_tok_off, i
                                       int chunk, int64_t* __restrict__ doc_chunk_off) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t carry;
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   if (tid == 0) {
     carry = 0;
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(PoolArgs a) {
     cw[j] = (float)c;
     sw[j] = (float)s;
   }
+  pdl_wait();  // the rotation constants above overlapped the previous kernel's tail
+  pdl_trigger();
 
   for (int64_t c = blockIdx.x; c < a.n_chunks; c += gridDim.x) {
     if (tid == 0) {
@@ -232,6 +236,8 @@ __global__ void bank_norms_kernel(const uint16_t* __restrict__ kbar_r, int64_t n
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int pairs = (hr + 1) / 2;
+  pdl_wait();
+  pdl_trigger();
   for (int64_t c = warp; c < n_chunks; c += n_warps) {
     for (int i = 0; i < pairs; ++i) {
       int h = 2 * i + (lane >> 4);
@@ -256,7 +262,9 @@ __global__ void bank_norms_kernel(const uint16_t* __restrict__ kbar_r, int64_t n
 }  // namespace
 
 msa_status launch_encode(const msa_encode_args& a, cudaStream_t st) {
-  doc_chunk_scan_kernel<<<1, 1024, 0, st>>>(a.doc_tok_off, a.n_docs, a.chunk, a.doc_chunk_off);
+  cudaError_t e = launch_pdl(doc_chunk_scan_kernel, dim3(1), dim3(1024), 0, st, a.doc_tok_off, a.n_docs, a.chunk,
+                             a.doc_chunk_off);
+  if (e != cudaSuccess) return cuda_fail(e, "encode: document index");
   msa_status s = launch_check("encode: document index");
   if (s != MSA_OK || a.n_chunks == 0) return s;
   PoolArgs p;
@@ -272,7 +280,8 @@ msa_status launch_encode(const msa_encode_args& a, cudaStream_t st) {
   int threads = 32 * ((heads + 1) / 2);  // whole warps: the norm reduction shuffles full warps
   int64_t grid = a.n_chunks < 148 * 40 ? a.n_chunks : 148 * 40;
   record_debug_event(0, st);
-  encode_pool_kernel<<<(unsigned)grid, threads, 0, st>>>(p);
+  e = launch_pdl(encode_pool_kernel, dim3((unsigned)grid), dim3(threads), 0, st, p);
+  if (e != cudaSuccess) return cuda_fail(e, "encode: pooling");
   msa_status s2 = launch_check("encode: pooling");
   record_debug_event(1, st);
   return s2;
@@ -284,7 +293,9 @@ msa_status launch_bank_norms(const uint16_t* kbar_r, int64_t n_chunks, int hr, f
   int64_t warps = n_chunks;
   int64_t blocks = (warps * 32 + 255) / 256;
   if (blocks > 148 * 32) blocks = 148 * 32;
-  bank_norms_kernel<<<(unsigned)blocks, 256, 0, st>>>(kbar_r, n_chunks, hr, eps, inv_norm);
+  cudaError_t e = launch_pdl(bank_norms_kernel, dim3((unsigned)blocks), dim3(256), 0, st, kbar_r, n_chunks, hr, eps,
+                             inv_norm);
+  if (e != cudaSuccess) return cuda_fail(e, "bank norms");
   return launch_check("bank norms");
 }
 

@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(1024) gather_index_kernel(
     int k, int64_t* __restrict__ sel_off, int64_t* __restrict__ sel_chunk) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t carry;
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int64_t n_pairs = (int64_t)n_seq * k;
   if (tid == 0) carry = 0;
@@ -69,6 +71,8 @@ __global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint
                                    const int64_t* __restrict__ sel_total,
                                    const int64_t* __restrict__ sel_chunk, int64_t cap, int hkv,
                                    uint16_t* __restrict__ stage_k, uint16_t* __restrict__ stage_v) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -106,7 +110,9 @@ __global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint
 
 msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
                                int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st) {
-  gather_index_kernel<<<1, 1024, 0, st>>>(b.doc_chunk_off, top_ids, n_seq, k, sel_off, sel_chunk);
+  cudaError_t e = launch_pdl(gather_index_kernel, dim3(1), dim3(1024), 0, st, b.doc_chunk_off, top_ids, n_seq, k,
+                             sel_off, sel_chunk);
+  if (e != cudaSuccess) return cuda_fail(e, "gather: chunk list");
   return launch_check("gather: chunk list");
 }
 
@@ -117,8 +123,9 @@ msa_status launch_gather_pull(const msa_bank_layer& b, const int64_t* sel_off, c
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
   // sel_off[n_seq] is the total row count; the caller passes its address.
-  gather_pull_kernel<<<(unsigned)blocks, 256, 0, st>>>(b.kbar, b.vbar, sel_off, sel_chunk, cap, b.hkv,
-                                                       stage_k, stage_v);
+  cudaError_t e = launch_pdl(gather_pull_kernel, dim3((unsigned)blocks), dim3(256), 0, st, b.kbar, b.vbar, sel_off,
+                             sel_chunk, cap, b.hkv, stage_k, stage_v);
+  if (e != cudaSuccess) return cuda_fail(e, "gather: device pull from host memory");
   return launch_check("gather: device pull from host memory");
 }
 

@@ -224,8 +224,8 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   for (int i = 0; i <= n_seq; ++i) p.q_seq_off[i] = q_seq_off[i];
   p.invq = reinterpret_cast<float*>(w + L.invq);
   p.doc_key = reinterpret_cast<uint32_t*>(w + L.doc_key);
-  cudaError_t e = cudaMemsetAsync(w + L.doc_key, 0, L.total - L.doc_key, st);
-  if (e != cudaSuccess) return cuda_fail(e, "route: clear workspace");
+  p.zero = w + L.doc_key;
+  p.zero_bytes = L.total - L.doc_key;  // a multiple of 256
   s = launch_qprep(p, eps, st);
   if (s != MSA_OK) return s;
   if (b->n_chunks > 0) {

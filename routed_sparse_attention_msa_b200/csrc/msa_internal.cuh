@@ -18,6 +18,32 @@ void record_debug_event(int which, cudaStream_t st);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// ------------------------------------------------ programmatic dependent launch
+// Every kernel of the path is launched so that it may start while its
+// predecessor on the stream is still finishing. Each kernel calls pdl_wait()
+// before it reads or writes any memory that another kernel touches (that wait
+// returns once the predecessor, and transitively everything before it, has
+// completed and its writes are visible), then pdl_trigger() so that its own
+// successor can be scheduled. Launched without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kHeadDim = 128;
 constexpr int kMaxSeq = 256;
 
@@ -74,6 +100,8 @@ struct RoutePlan {
   int32_t q_seq_off[kMaxSeq + 1];
   float* invq;                 // ws [T, hr]: 1 / (hr * max(||q||, eps))
   uint32_t* doc_key;           // ws [S, D]: ordered doc scores (0 = none)
+  void* zero;                  // ws bytes to clear before scoring (doc keys, top-k state)
+  size_t zero_bytes;           // multiple of 16
 };
 
 // score.cu

@@ -20,11 +20,16 @@
 namespace msa {
 namespace {
 
-// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)).
+// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)); the whole grid
+// also clears the scoring workspace (document keys and top-k state).
 __global__ void qprep_kernel(const uint16_t* __restrict__ qr, int n_rows, int hr, float eps,
-                             float* __restrict__ invq) {
+                             float* __restrict__ invq, uint4* __restrict__ zero, int64_t zero_vecs) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < zero_vecs; i += (int64_t)gridDim.x * blockDim.x) zero[i] = make_uint4(0, 0, 0, 0);
   const int lane = threadIdx.x & 31;
-  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int w = (int)(tid >> 5);
   if (w >= n_rows * hr) return;
   uint2 v = __ldg(reinterpret_cast<const uint2*>(qr + (size_t)w * kHeadDim + 4 * lane));
   float a = bf_lo(v.x), b = bf_hi(v.x), c = bf_lo(v.y), d = bf_hi(v.y);
@@ -52,6 +57,8 @@ constexpr int kChunksPerWarpTask = 64;
 
 template <int TP>
 __global__ void __launch_bounds__(256) score_simt_kernel(SimtArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -143,9 +150,14 @@ __global__ void __launch_bounds__(256) score_simt_kernel(SimtArgs a) {
 }  // namespace
 
 msa_status launch_qprep(const RoutePlan& p, float eps, cudaStream_t st) {
-  int warps = p.n_rows * p.hr;
-  int blocks = (warps * 32 + 255) / 256;
-  qprep_kernel<<<blocks, 256, 0, st>>>(p.qr, p.n_rows, p.hr, eps, p.invq);
+  const int64_t warps = (int64_t)p.n_rows * p.hr;
+  int64_t blocks = (warps * 32 + 255) / 256;
+  const int64_t zvecs = (int64_t)(p.zero_bytes / 16);
+  const int64_t zblocks = (zvecs + 255) / 256;
+  if (blocks < zblocks) blocks = zblocks < 148 * 4 ? zblocks : 148 * 4;
+  cudaError_t e = launch_pdl(qprep_kernel, dim3((unsigned)blocks), dim3(256), 0, st, p.qr, p.n_rows, p.hr, eps,
+                             p.invq, reinterpret_cast<uint4*>(p.zero), zvecs);
+  if (e != cudaSuccess) return cuda_fail(e, "route: query norms");
   return launch_check("route: query norms");
 }
 

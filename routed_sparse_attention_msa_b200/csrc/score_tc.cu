@@ -210,6 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the prologue above overlapped the previous kernel's tail
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
@@ -448,7 +450,8 @@ msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int grid = a.n_tiles < sms ? a.n_tiles : sms;
-  score_tc_kernel<NB><<<grid, kThreads, C::kSmem, st>>>(mk, mq, a);
+  cudaError_t e = launch_pdl(score_tc_kernel<NB>, dim3(grid), dim3(kThreads), (size_t)C::kSmem, st, mk, mq, a);
+  if (e != cudaSuccess) return cuda_fail(e, "route: score (tensor cores)");
   return launch_check("route: score (tensor cores)");
 }
 

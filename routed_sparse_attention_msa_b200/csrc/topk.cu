@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(
     float* __restrict__ all_scores) {
   __shared__ uint64_t s_lists[kWarps][32];
   __shared__ bool s_last;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int s = blockIdx.y;
   const int part = blockIdx.x;
@@ -151,6 +153,8 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
     float* __restrict__ all_scores) {
   __shared__ uint64_t s_lists[kWarps][16];
   __shared__ bool s_last;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int s = blockIdx.y;
   const int part = blockIdx.x;
@@ -214,6 +218,8 @@ __global__ void __launch_bounds__(1024) topk_radix_kernel(
   __shared__ uint64_t s_prefix, s_mask;
   __shared__ int s_krem;
   __shared__ unsigned s_count;
+  pdl_wait();
+  pdl_trigger();
   const int s = blockIdx.x;
   const uint32_t* keys = doc_key + (size_t)s * n_docs;
   const int tid = threadIdx.x;
@@ -304,14 +310,10 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
     unsigned* tickets = reinterpret_cast<unsigned*>(
         reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256));
     dim3 grid((unsigned)parts, (unsigned)n_seq);
-    if (k <= 16) {
-      topk16_kernel<<<grid, kWarps * 32, 0, st>>>(doc_key, n_docs, k, cand, tickets, top_ids, top_scores,
-                                                  all_scores);
-      return launch_check("route: top-k (bitonic, k <= 16)");
-    }
-    topk_warp_kernel<<<grid, kWarps * 32, 0, st>>>(doc_key, n_docs, k, cand, tickets, top_ids,
-                                                   top_scores, all_scores);
-    return launch_check("route: top-k (warp insertion)");
+    cudaError_t e = launch_pdl(k <= 16 ? topk16_kernel : topk_warp_kernel, grid, dim3(kWarps * 32), 0, st,
+                               doc_key, n_docs, k, cand, tickets, top_ids, top_scores, all_scores);
+    if (e != cudaSuccess) return cuda_fail(e, "route: top-k");
+    return launch_check("route: top-k");
   }
   int pow2 = 1;
   while (pow2 < k) pow2 <<= 1;
@@ -321,7 +323,9 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
                                          (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "route: top-k shared memory");
   }
-  topk_radix_kernel<<<n_seq, 1024, smem, st>>>(doc_key, n_docs, k, top_ids, top_scores, all_scores);
+  cudaError_t e = launch_pdl(topk_radix_kernel, dim3(n_seq), dim3(1024), smem, st, doc_key, n_docs, k, top_ids,
+                             top_scores, all_scores);
+  if (e != cudaSuccess) return cuda_fail(e, "route: top-k (radix)");
   return launch_check("route: top-k (radix)");
 }
 
