@@ -104,7 +104,9 @@ typedef struct msa_bank_layer {
  *
  * Document j is tokens doc_tok_off[j] .. doc_tok_off[j+1]-1 of the per-token
  * arrays. For every token at document-local position p, K is rotated by RoPE
- * at position p (half-split pairs (i, i + d/2), angle p * rope_theta^(-2i/d)).
+ * at position p (half-split pairs (i, i + d/2), angle p * rope_theta^(-2i/d));
+ * with rope_mode = 1 the rotation is instead applied to each pooled chunk at
+ * its chunk index within the document (the pages leave the order open).
  * Each document is cut into chunks of `chunk` tokens (the last may be
  * shorter; chunks never cross documents) and K, V, K_r are averaged over the
  * tokens of each chunk, in fp32, rounded to bf16 (nearest even). The inverse
@@ -128,6 +130,10 @@ typedef struct msa_encode_args {
   float* kr_inv_norm;           /* device out [n_chunks, hr] */
   int64_t* doc_chunk_off;       /* device out [n_docs + 1] */
   int32_t* chunk_doc;           /* device out [n_chunks] */
+  int32_t rope_mode;            /* 0: rotate each token at its document-local position, then pool
+                                   (default reading); 1: pool, then rotate each pooled chunk at its
+                                   chunk index within the document (alternative reading) */
+  int32_t reserved;
 } msa_encode_args;
 
 /* Host-side planning: n_chunks = sum_j ceil(len_j / chunk) from a HOST copy
@@ -171,6 +177,27 @@ msa_status msa_route(const msa_bank_layer* bank, const uint16_t* qr, const int32
                      int32_t n_seq, int32_t n_rows, int32_t top_k, float eps,
                      int32_t* top_ids, float* top_scores, float* all_doc_scores,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Merge of per-shard top-k lists (Memory Parallel).
+ *
+ * ["MSA: Memory Sparse Attention", Inference Pipeline: Memory Parallel shards
+ * the routing keys across GPUs — query broadcast, local scoring, global
+ * reduce; "MSA-arXiv26", 核心方法 / Memory Parallel inference]
+ *
+ * When the documents are split into n_shards contiguous ranges, each routed
+ * by msa_route on its own bank (local document ids), shard g's lists
+ * ids[g, s, :] / scores[g, s, :] (device, [n_shards, n_seq, k]) hold its
+ * best k documents of sequence s; id_offset[g] (HOST) is the global id of its
+ * first document. The merge writes the best k_out of all shards' candidates
+ * (k_out <= n_shards * k) in the same order as msa_route on the whole bank
+ * (score descending, then global id ascending), so the result is identical
+ * to routing the unsharded bank. Entries with id < 0 are ignored.
+ * Limits: n_shards <= 64, n_shards * k <= 4096.
+ * ---------------------------------------------------------------------- */
+msa_status msa_topk_merge(const int32_t* ids, const float* scores, const int64_t* id_offset,
+                          int32_t n_shards, int32_t n_seq, int32_t k, int32_t k_out,
+                          int32_t* top_ids, float* top_scores, void* stream);
 
 /* ------------------------------------------------------------------------
  * Route without a workspace. The pages have no counterpart: this is an

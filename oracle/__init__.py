@@ -73,7 +73,7 @@ def _load():
         lib.orc_double_array_to_bf16.restype = None
         lib.orc_rope.argtypes = [P, i32, f64, f64]
         lib.orc_rope.restype = i32
-        lib.orc_encode.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, f64, f64,
+        lib.orc_encode.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, f64, f64, i32,
                                    P, P, P, P, P, P, i64]
         lib.orc_encode.restype = i32
         lib.orc_route.argtypes = [P, P, i64, i32, i32, P, P, i32, f64, i32, P, P, P]
@@ -128,9 +128,10 @@ def rope(x: np.ndarray, pos: float, theta: float) -> np.ndarray:
 
 # ------------------------------------------------------------------- encode
 
-def encode(k_tok, v_tok, kr_tok, doc_tok_off, chunk=64, rope_theta=1e6, eps=1e-8):
+def encode(k_tok, v_tok, kr_tok, doc_tok_off, chunk=64, rope_theta=1e6, eps=1e-8, rope_mode=0):
     """Offline encode of one layer. Per-token arrays are uint16 bfloat16 bits
-    shaped [n_tok, heads, d]. Returns a dict of pooled outputs."""
+    shaped [n_tok, heads, d]. rope_mode 0 rotates tokens before pooling, 1
+    rotates the pooled chunk at its chunk index. Returns the pooled outputs."""
     k_tok, v_tok, kr_tok = _u16(k_tok), _u16(v_tok), _u16(kr_tok)
     off = np.ascontiguousarray(doc_tok_off, dtype=np.int64)
     n_docs = off.size - 1
@@ -145,7 +146,7 @@ def encode(k_tok, v_tok, kr_tok, doc_tok_off, chunk=64, rope_theta=1e6, eps=1e-8
     dco = np.empty(n_docs + 1, np.int64)
     cdoc = np.empty(max(n_chunks, 1), np.int32)
     rc = _load().orc_encode(_p(k_tok), _p(v_tok), _p(kr_tok), _p(off), n_docs, hkv, hr, d,
-                            chunk, float(rope_theta), float(eps), _p(kbar), _p(vbar), _p(kbar_r),
+                            chunk, float(rope_theta), float(eps), int(rope_mode), _p(kbar), _p(vbar), _p(kbar_r),
                             _p(inv), _p(dco), _p(cdoc), n_chunks)
     if rc != 0:
         raise ValueError(f"orc_encode failed ({rc})")

@@ -82,10 +82,11 @@ int orc_rope(double* x, int d, double pos, double theta) {
  *    routing key is taken from the stored (rounded) values, clamped at eps. */
 int orc_encode(const uint16_t* k_tok, const uint16_t* v_tok, const uint16_t* kr_tok,
                const int64_t* doc_tok_off, int64_t n_docs, int hkv, int hr, int d, int chunk,
-               double rope_theta, double eps,
+               double rope_theta, double eps, int rope_mode,
                uint16_t* kbar, uint16_t* vbar, uint16_t* kbar_r, double* kr_inv_norm,
                int64_t* doc_chunk_off, int32_t* chunk_doc, int64_t n_chunks) {
   if (n_docs < 0 || hkv <= 0 || hr <= 0 || d <= 0 || (d & 1) || chunk <= 0) return -1;
+  if (rope_mode != 0 && rope_mode != 1) return -1;
   int64_t total = 0;
   for (int64_t j = 0; j < n_docs; ++j) {
     int64_t len = doc_tok_off[j + 1] - doc_tok_off[j];
@@ -121,7 +122,7 @@ int orc_encode(const uint16_t* k_tok, const uint16_t* v_tok, const uint16_t* kr_
         for (int h = 0; h < hkv; ++h) {
           const uint16_t* src = k_tok + ((size_t)t * hkv + h) * d;
           for (int i = 0; i < d; ++i) row[i] = orc_bf16_to_double(src[i]);
-          orc_rope(row, d, (double)p, rope_theta);
+          if (rope_mode == 0) orc_rope(row, d, (double)p, rope_theta);
           for (int i = 0; i < d; ++i) sk[(size_t)h * d + i] += row[i];
           const uint16_t* vs = v_tok + ((size_t)t * hkv + h) * d;
           for (int i = 0; i < d; ++i) sv[(size_t)h * d + i] += orc_bf16_to_double(vs[i]);
@@ -131,6 +132,8 @@ int orc_encode(const uint16_t* k_tok, const uint16_t* v_tok, const uint16_t* kr_
           for (int i = 0; i < d; ++i) sr[(size_t)h * d + i] += orc_bf16_to_double(rs[i]);
         }
       }
+      if (rope_mode == 1) /* pooled chunk rotated at its chunk index */
+        for (int h = 0; h < hkv; ++h) orc_rope(sk + (size_t)h * d, d, (double)q, rope_theta);
       for (int64_t i = 0; i < (int64_t)hkv * d; ++i) {
         kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)n);
         vbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sv[i] / (double)n);

@@ -43,9 +43,13 @@ int orc_rope(double* x, int d, double pos, double theta);
  * C must equal sum_j ceil(len_j / chunk). */
 int orc_encode(const uint16_t* k_tok, const uint16_t* v_tok, const uint16_t* kr_tok,
                const int64_t* doc_tok_off, int64_t n_docs, int hkv, int hr, int d, int chunk,
-               double rope_theta, double eps,
+               double rope_theta, double eps, int rope_mode,
                uint16_t* kbar, uint16_t* vbar, uint16_t* kbar_r, double* kr_inv_norm,
                int64_t* doc_chunk_off, int32_t* chunk_doc, int64_t n_chunks);
+/* rope_mode 0: each token of K rotated at its document-local position, then
+ * pooled (the reading the library uses by default). rope_mode 1: K pooled
+ * first, the pooled chunk rotated at its chunk index within the document (an
+ * alternative reading of the same passage). */
 
 /* Online routing of one layer ([P2] Architecture; [P1] 核心方法):
  * cosine similarity of every query routing vector with every pooled routing

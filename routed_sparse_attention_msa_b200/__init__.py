@@ -51,7 +51,7 @@ class EncodeArgsC(ctypes.Structure):
     _fields_ = [("k_tok", P), ("v_tok", P), ("kr_tok", P), ("doc_tok_off", P), ("n_docs", i64),
                 ("n_tok", i64), ("n_chunks", i64), ("hkv", i32), ("hr", i32), ("d", i32), ("chunk", i32),
                 ("rope_theta", f32), ("eps", f32), ("kbar", P), ("vbar", P), ("kbar_r", P),
-                ("kr_inv_norm", P), ("doc_chunk_off", P), ("chunk_doc", P)]
+                ("kr_inv_norm", P), ("doc_chunk_off", P), ("chunk_doc", P), ("rope_mode", i32), ("reserved", i32)]
 
 
 class GatherArgsC(ctypes.Structure):
@@ -89,13 +89,14 @@ _sig("msa_bank_norms", [P, i64, i32, i32, f32, P, P])
 _sig("msa_route_workspace", [ctypes.POINTER(BankLayerC), i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)])
 _sig("msa_route", [ctypes.POINTER(BankLayerC), P, P, i32, i32, i32, f32, P, P, P, P, ctypes.c_size_t, P])
 _sig("msa_route_static", [ctypes.POINTER(BankLayerC), P, P, i32, i32, i32, f32, P, P, P, P])
+_sig("msa_topk_merge", [P, P, P, i32, i32, i32, i32, P, P, P])
 _sig("msa_gather", [ctypes.POINTER(GatherArgsC), P])
 _sig("msa_attend_workspace", [ctypes.POINTER(AttendArgsC), ctypes.POINTER(ctypes.c_size_t)])
 _sig("msa_attend", [ctypes.POINTER(AttendArgsC), P, ctypes.c_size_t, P])
 _sig("msa_sync_check", [P])
 
 EXPORTS = ["msa_status_string", "msa_last_error", "msa_version", "msa_encode_plan", "msa_encode",
-           "msa_bank_norms", "msa_route_workspace", "msa_route", "msa_route_static", "msa_gather", "msa_attend_workspace",
+           "msa_bank_norms", "msa_route_workspace", "msa_route", "msa_route_static", "msa_topk_merge", "msa_gather", "msa_attend_workspace",
            "msa_attend", "msa_sync_check"]
 
 
@@ -164,14 +165,14 @@ def encode_plan(doc_tok_off_host, chunk: int = 64):
 
 
 def encode(k_tok, v_tok, kr_tok, doc_tok_off, n_chunks: int, out: dict, chunk: int = 64,
-           rope_theta: float = 1e6, eps: float = 1e-8, stream=None) -> None:
+           rope_theta: float = 1e6, eps: float = 1e-8, rope_mode: int = 0, stream=None) -> None:
     """Encode one layer. Per-token tensors [n_tok, heads, 128] bf16 on the device,
     doc_tok_off int64 device; ``out`` holds device tensors kbar, vbar, kbar_r,
     kr_inv_norm, doc_chunk_off, chunk_doc."""
     a = EncodeArgsC(_ptr(k_tok), _ptr(v_tok), _ptr(kr_tok), _ptr(doc_tok_off), doc_tok_off.numel() - 1,
                     k_tok.shape[0], n_chunks, k_tok.shape[1], kr_tok.shape[1], k_tok.shape[2], chunk,
                     rope_theta, eps, _ptr(out["kbar"]), _ptr(out["vbar"]), _ptr(out["kbar_r"]),
-                    _ptr(out["kr_inv_norm"]), _ptr(out["doc_chunk_off"]), _ptr(out["chunk_doc"]))
+                    _ptr(out["kr_inv_norm"]), _ptr(out["doc_chunk_off"]), _ptr(out["chunk_doc"]), rope_mode, 0)
     _check(_lib.msa_encode(ctypes.byref(a), _stream(stream)), "msa_encode")
 
 
@@ -223,6 +224,16 @@ def route(bank: BankLayer, qr, q_seq_off_host, top_k: int, top_ids, top_scores, 
     _check(_lib.msa_route(ctypes.byref(b), _ptr(qr), qso.ctypes.data, qso.size - 1, qr.shape[0], top_k, eps,
                           _ptr(top_ids), _ptr(top_scores), _ptr(all_doc_scores), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream)), "msa_route")
+
+
+def topk_merge(ids, scores, id_offset_host, k_out: int, top_ids, top_scores, stream=None) -> None:
+    """Merge per-shard top-k lists ids/scores [G, S, k] (device; local ids, -1 =
+    padding) with each shard's first global document id (host [G]) into the
+    global top-k_out [S, k_out]."""
+    G, S, k = ids.shape
+    off = np.ascontiguousarray(np.asarray(id_offset_host, dtype=np.int64))
+    _check(_lib.msa_topk_merge(_ptr(ids), _ptr(scores), off.ctypes.data, G, S, k, k_out, _ptr(top_ids),
+                               _ptr(top_scores), _stream(stream)), "msa_topk_merge")
 
 
 ROUTE_STATIC_SCRATCH_BYTES = 4 << 20  # MSA_ROUTE_STATIC_SCRATCH_BYTES

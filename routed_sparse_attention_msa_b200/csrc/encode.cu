@@ -77,7 +77,7 @@ struct PoolArgs {
   const int64_t* doc_tok_off;
   const int64_t* doc_chunk_off;
   int64_t n_docs, n_chunks;
-  int hkv, hr, chunk;
+  int hkv, hr, chunk, rope_mode;
   double log2_theta;
   float eps;
   uint16_t* kbar;
@@ -97,7 +97,7 @@ __device__ __forceinline__ void acc8(float* s, uint4 w) {
 constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(256) encode_pool_kernel(PoolArgs a) {
-  __shared__ int64_t s_t0, s_p0;
+  __shared__ int64_t s_t0, s_p0;  // first token; rotation position of the pooled chunk
   __shared__ int s_n;
   const int tid = threadIdx.x;
   const int h = tid >> 4;   // head owned by this thread
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(PoolArgs a) {
       int64_t t0 = a.doc_tok_off[lo] + q * a.chunk;
       int64_t len = a.doc_tok_off[lo + 1] - t0;
       s_t0 = t0;
-      s_p0 = q * a.chunk;
+      s_p0 = a.rope_mode == 1 ? q : q * a.chunk;
       s_n = (int)(len < a.chunk ? len : a.chunk);
       a.chunk_doc[c] = (int32_t)lo;
     }
@@ -173,13 +173,22 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(PoolArgs a) {
           float x0[4] = {bf_lo(kl[e].x), bf_hi(kl[e].x), bf_lo(kl[e].y), bf_hi(kl[e].y)};
           float x1[4] = {bf_lo(kh[e].x), bf_hi(kh[e].x), bf_lo(kh[e].y), bf_hi(kh[e].y)};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ka[j] += x0[j] * cr[j] - x1[j] * sr[j];
-            kb[j] += x0[j] * sr[j] + x1[j] * cr[j];
-            float c2 = cr[j] * cw[j] - sr[j] * sw[j];
-            float s2 = sr[j] * cw[j] + cr[j] * sw[j];
-            cr[j] = c2;
-            sr[j] = s2;
+          if (a.rope_mode == 1) {  // pool first; the chunk is rotated below
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              ka[j] += x0[j];
+              kb[j] += x1[j];
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              ka[j] += x0[j] * cr[j] - x1[j] * sr[j];
+              kb[j] += x0[j] * sr[j] + x1[j] * cr[j];
+              float c2 = cr[j] * cw[j] - sr[j] * sw[j];
+              float s2 = sr[j] * cw[j] + cr[j] * sw[j];
+              cr[j] = c2;
+              sr[j] = s2;
+            }
           }
           acc8(vs, vv[e]);
           acc8(rs, rr[e]);
@@ -271,7 +280,7 @@ msa_status launch_encode(const msa_encode_args& a, cudaStream_t st) {
   p.k_tok = a.k_tok; p.v_tok = a.v_tok; p.kr_tok = a.kr_tok;
   p.doc_tok_off = a.doc_tok_off; p.doc_chunk_off = a.doc_chunk_off;
   p.n_docs = a.n_docs; p.n_chunks = a.n_chunks;
-  p.hkv = a.hkv; p.hr = a.hr; p.chunk = a.chunk;
+  p.hkv = a.hkv; p.hr = a.hr; p.chunk = a.chunk; p.rope_mode = a.rope_mode;
   p.log2_theta = log2((double)a.rope_theta);
   p.eps = a.eps;
   p.kbar = a.kbar; p.vbar = a.vbar; p.kbar_r = a.kbar_r; p.inv_norm = a.kr_inv_norm;

@@ -168,6 +168,7 @@ msa_status msa_encode(const msa_encode_args* a, void* stream) {
   if (a->n_docs <= 0 || a->n_tok < 0 || a->n_chunks < 0) return fail(MSA_ERR_INVALID_ARG, "encode: bad sizes");
   if (!(a->rope_theta > 1.0f) || !(a->eps > 0.0f)) return fail(MSA_ERR_INVALID_ARG, "encode: rope_theta > 1 and eps > 0 required");
   if (!a->doc_tok_off || !a->doc_chunk_off) return fail(MSA_ERR_INVALID_ARG, "encode: NULL offsets");
+  if (a->rope_mode != 0 && a->rope_mode != 1) return fail(MSA_ERR_INVALID_ARG, "encode: rope_mode = %d", a->rope_mode);
   if (a->n_chunks > 0 && (!a->k_tok || !a->v_tok || !a->kr_tok || !a->kbar || !a->vbar || !a->kbar_r ||
                           !a->kr_inv_norm || !a->chunk_doc))
     return fail(MSA_ERR_INVALID_ARG, "encode: NULL tensor");
@@ -238,6 +239,19 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   }
   int k = top_k < b->n_docs ? top_k : (int)b->n_docs;
   return launch_topk(p.doc_key, n_seq, b->n_docs, k, top_ids, top_scores, all_doc_scores, w + L.topk, st);
+}
+
+msa_status msa_topk_merge(const int32_t* ids, const float* scores, const int64_t* id_offset, int32_t n_shards,
+                          int32_t n_seq, int32_t k, int32_t k_out, int32_t* top_ids, float* top_scores,
+                          void* stream) {
+  if (!ids || !scores || !id_offset || !top_ids || !top_scores) return fail(MSA_ERR_INVALID_ARG, "topk_merge: NULL pointer");
+  if (n_seq <= 0 || n_seq > 65535 || k <= 0 || k_out <= 0 || k_out > n_shards * k)
+    return fail(MSA_ERR_INVALID_ARG, "topk_merge: bad sizes");
+  if ((int64_t)n_shards * k > 4096) return fail(MSA_ERR_UNSUPPORTED, "topk_merge: n_shards * k > 4096");
+  for (int g = 0; g < n_shards && g < 64; ++g)
+    if (id_offset[g] < 0 || id_offset[g] > 0x7FFFFFFF) return fail(MSA_ERR_INVALID_ARG, "topk_merge: id_offset[%d]", g);
+  return launch_topk_merge(ids, scores, id_offset, n_shards, n_seq, k, k_out, top_ids, top_scores,
+                           (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ gather

@@ -119,6 +119,9 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
                        int32_t* top_ids, float* top_scores, float* all_scores, void* ws,
                        cudaStream_t st);
 
+msa_status launch_topk_merge(const int32_t* ids, const float* scores, const int64_t* id_offset, int n_shards,
+                             int n_seq, int k, int k_out, int32_t* top_ids, float* top_scores, cudaStream_t st);
+
 // gather.cu
 msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
                                int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st);

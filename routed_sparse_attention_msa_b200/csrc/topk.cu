@@ -289,7 +289,82 @@ __global__ void __launch_bounds__(1024) topk_radix_kernel(
     write_result(s_sel[i], top_ids + (size_t)s * k + i, top_scores + (size_t)s * k + i);
 }
 
+// Merge of per-shard top-k lists (Memory Parallel): one CTA per sequence
+// loads every shard's k (score, local id) pairs, forms the global keys with
+// the shard's document offset, sorts them (bitonic, descending) in shared
+// memory and keeps the best k. Entries with a negative id are padding.
+constexpr int kMaxShards = 64;
+struct MergeArgs {
+  const int32_t* ids;    // [G, S, k]
+  const float* scores;   // [G, S, k]
+  int32_t* top_ids;      // [S, k_out]
+  float* top_scores;     // [S, k_out]
+  int n_shards, n_seq, k, k_out, pow2;
+  int64_t id_offset[kMaxShards];
+};
+
+__global__ void __launch_bounds__(1024) topk_merge_kernel(const __grid_constant__ MergeArgs a) {
+  extern __shared__ uint64_t s_keys[];  // [pow2]
+  pdl_wait();
+  pdl_trigger();
+  const int s = blockIdx.x, tid = threadIdx.x;
+  const int n = a.n_shards * a.k;
+  for (int i = tid; i < a.pow2; i += blockDim.x) {
+    uint64_t key = 0;
+    if (i < n) {
+      const int g = i / a.k, j = i % a.k;
+      const size_t src = ((size_t)g * a.n_seq + s) * a.k + j;
+      const int32_t id = a.ids[src];
+      if (id >= 0) {
+        const float sc = a.scores[src];
+        const uint32_t o = __float_as_uint(sc) == 0xff800000u ? 0u : ord_f32(sc);  // -inf: never scored
+        key = doc_key64(o, (int64_t)id + a.id_offset[g]);
+      }
+    }
+    s_keys[i] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= a.pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < a.pow2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const uint64_t x = s_keys[i], y = s_keys[j];
+          if (desc ? (x < y) : (x > y)) {
+            s_keys[i] = y;
+            s_keys[j] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < a.k_out; i += blockDim.x)
+    write_result(s_keys[i], a.top_ids + (size_t)s * a.k_out + i, a.top_scores + (size_t)s * a.k_out + i);
+}
+
 }  // namespace
+
+msa_status launch_topk_merge(const int32_t* ids, const float* scores, const int64_t* id_offset, int n_shards,
+                             int n_seq, int k, int k_out, int32_t* top_ids, float* top_scores, cudaStream_t st) {
+  if (n_shards <= 0 || n_shards > kMaxShards) return fail(MSA_ERR_UNSUPPORTED, "topk_merge: %d shards (1..%d)", n_shards, kMaxShards);
+  MergeArgs a{};
+  a.ids = ids; a.scores = scores; a.top_ids = top_ids; a.top_scores = top_scores;
+  a.n_shards = n_shards; a.n_seq = n_seq; a.k = k; a.k_out = k_out;
+  int pow2 = 1;
+  while (pow2 < n_shards * k) pow2 <<= 1;
+  a.pow2 = pow2;
+  for (int g = 0; g < n_shards; ++g) a.id_offset[g] = id_offset[g];
+  const size_t smem = (size_t)pow2 * sizeof(uint64_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "topk_merge: shared memory");
+  }
+  cudaError_t e = launch_pdl(topk_merge_kernel, dim3(n_seq), dim3(1024), smem, st, a);
+  if (e != cudaSuccess) return cuda_fail(e, "topk_merge");
+  return launch_check("topk_merge");
+}
 
 size_t topk_workspace(int n_seq, int64_t n_docs, int k) {
   int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;

@@ -11,6 +11,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -60,3 +61,51 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--workload", "tiny", "--steps", "1", "--warmup", "0"], env=env, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _gather_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from routed_sparse_attention_msa_b200 import memory_parallel as mp
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ids = torch.full((3, 4), rank, dtype=torch.int32)
+        sc = torch.full((3, 4), 0.5 * rank, dtype=torch.float32)
+        all_ids, all_sc = mp.gather_candidates(ids, sc)
+        q.put((rank, all_ids.tolist(), all_sc.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_memory_parallel_candidate_gather_on_gloo():
+    """Every rank receives every rank's [S, k] candidates, stacked by rank."""
+    pytest.importorskip("routed_sparse_attention_msa_b200")
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for rank, ids, sc in sorted(q.get(timeout=10) for _ in range(world)):
+        assert [row[0][0] for row in ids] == [0, 1]
+        assert [row[0][0] for row in sc] == [0.0, 0.5]
+
+
+def test_shard_ranges_balance_chunks():
+    from routed_sparse_attention_msa_b200 import memory_parallel as mpar
+    import synth
+    dco, _ = synth.workload("10m").index()
+    r = mpar.shard_ranges(dco, 8)
+    assert r[0][0] == 0 and r[-1][1] == dco.size - 1
+    assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+    counts = [int(dco[b] - dco[a]) for a, b in r]
+    assert max(counts) - min(counts) <= 2 * int(np.diff(dco).max())
+    assert mpar.shard_ranges(np.array([0, 5, 5, 9]), 5)[-1] == (3, 3)  # more shards than documents

@@ -46,8 +46,8 @@ def test_device_generator_matches_host():
 ENC_LENS = [64, 1, 63, 65, 0, 129, 300, 4096 + 17, 640, 2]
 
 
-@pytest.mark.parametrize("theta", [1e6, 1e4])
-def test_encode_matches_oracle(msa, theta):
+@pytest.mark.parametrize("theta,rope_mode", [(1e6, 0), (1e4, 0), (1e4, 1)])
+def test_encode_matches_oracle(msa, theta, rope_mode):
     off = np.concatenate([[0], np.cumsum(ENC_LENS)]).astype(np.int64)
     n = int(off[-1])
     shp = (n, 8, 128)
@@ -61,10 +61,10 @@ def test_encode_matches_oracle(msa, theta):
                kr_inv_norm=torch.empty((C, 8), dtype=torch.float32, device="cuda"),
                doc_chunk_off=torch.empty(len(ENC_LENS) + 1, dtype=torch.int64, device="cuda"),
                chunk_doc=torch.empty(C, dtype=torch.int32, device="cuda"))
-    msa.encode(k, v, r, torch.from_numpy(off).cuda(), C, out, rope_theta=theta)
+    msa.encode(k, v, r, torch.from_numpy(off).cuda(), C, out, rope_theta=theta, rope_mode=rope_mode)
     msa.sync_check()
     ref = oracle.encode(host_normal(shp, synth.tid("k_tok", 1)), host_normal(shp, synth.tid("v_tok", 1)),
-                        host_normal(shp, synth.tid("kr_tok", 1)), off, rope_theta=theta)
+                        host_normal(shp, synth.tid("kr_tok", 1)), off, rope_theta=theta, rope_mode=rope_mode)
     np.testing.assert_array_equal(out["doc_chunk_off"].cpu().numpy(), ref["doc_chunk_off"])
     np.testing.assert_array_equal(out["doc_chunk_off"].cpu().numpy(), dco_h)
     np.testing.assert_array_equal(out["chunk_doc"].cpu().numpy(), ref["chunk_doc"])
@@ -266,6 +266,16 @@ def test_attend_matches_oracle(msa, case):
     err = np.abs(g_f32 - o_out).max()
     assert err <= 1e-2, err
     np.testing.assert_array_equal(g_out, synth.bf16_bits(g_f32))  # bf16 out = nearest-even of the fp32 result
+    np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
+
+
+def test_attend_block_length_offset_reading(msa):
+    """The alternative reading of the query offset: k retrieved documents x the
+    chunk length (pos_offset = 16 * 64) instead of k."""
+    c = _attend_case(rows=(2, 1), n_loc=(5, 70), n_mem=(48, 90), q_start=(3, 69), layer=22)
+    g_out, g_f32, g_lse = _attend_gpu(msa, c, 1024.0)
+    o_out, o_lse = oracle.attend(**c, pos_offset=1024.0)
+    assert np.abs(g_f32 - o_out).max() <= 1e-2
     np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
 
 

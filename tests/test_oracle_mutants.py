@@ -22,6 +22,8 @@ MUTANTS = {
     "rope_pairing": ("double x0 = x[i], x1 = x[i + h];", "double x0 = x[i], x1 = x[(i + h + 1) % d];"),
     "encode_global_position": ("int64_t p = q * chunk + u; /* document-local position */",
                                "int64_t p = t0 + q * chunk + u;"),
+    "encode_chunk_rotation_global": ("orc_rope(sk + (size_t)h * d, d, (double)q, rope_theta);",
+                                     "orc_rope(sk + (size_t)h * d, d, (double)c, rope_theta);"),
     "encode_full_chunk_divisor": ("kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)n);",
                                   "kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)chunk);"),
     "encode_norm_unrounded": ("double x = orc_bf16_to_double(b);", "double x = sr[(size_t)h * d + i] / (double)n + 1e-3;"),
