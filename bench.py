@@ -242,18 +242,25 @@ class Routed:
             self.vl_h.append(synth.normal_bf16_host(S * self.Lloc * hkv * d, synth.tid("v_loc", l)).reshape(
                 S * self.Lloc, hkv, d))
 
-        def up(a):
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        def up(arrs):  # all layers in one tensor; layer l is the contiguous view [l]
+            a = np.ascontiguousarray(np.stack(arrs))
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
 
-        self.qr_d = [up(a) for a in self.qr_h]
-        self.q_d = [up(a) for a in self.q_h]
-        self.kl_d = [up(a) for a in self.kl_h]
-        self.vl_d = [up(a) for a in self.vl_h]
+        self.qr_all = up(self.qr_h)
+        self.q_all = up(self.q_h)
+        self.kl_all = up(self.kl_h)
+        self.vl_all = up(self.vl_h)
+        self.qr_d = [self.qr_all[l] for l in range(self.L)]
+        self.q_d = [self.q_all[l] for l in range(self.L)]
+        self.kl_d = [self.kl_all[l] for l in range(self.L)]
+        self.vl_d = [self.vl_all[l] for l in range(self.L)]
         # outputs and workspaces (shared by layers; the stream orders their reuse)
         kk = min(k, w.n_docs)
         self.kk = kk
-        self.ids = [torch.empty((S, kk), dtype=torch.int32, device="cuda") for _ in range(self.L)]
-        self.scores = [torch.empty((S, kk), dtype=torch.float32, device="cuda") for _ in range(self.L)]
+        self.ids_all = torch.empty((self.L, S, kk), dtype=torch.int32, device="cuda")
+        self.scores_all = torch.empty((self.L, S, kk), dtype=torch.float32, device="cuda")
+        self.ids = [self.ids_all[l] for l in range(self.L)]
+        self.scores = [self.scores_all[l] for l in range(self.L)]
         self.ws_route = torch.empty(msa.route_workspace(self.banks[0], S, self.T, k), dtype=torch.uint8, device="cuda")
         self.cap = S * kk * self.max_doc_chunks
         self.sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
@@ -265,7 +272,8 @@ class Routed:
             self.copy_stream = torch.cuda.Stream()
             self.copy_done = torch.cuda.Event()
             self.copy_done.record(self.copy_stream)
-        self.out = [torch.empty((self.Tq, w.hq, d), dtype=torch.bfloat16, device="cuda") for _ in range(self.L)]
+        self.out_all = torch.empty((self.L, self.Tq, w.hq, d), dtype=torch.bfloat16, device="cuda")
+        self.out = [self.out_all[l] for l in range(self.L)]
         self.pos_offset = float(k)
         a0 = self._attend_args(0)
         self.ws_attend = torch.empty(msa.attend_workspace(*a0, pos_offset=self.pos_offset, rope_theta=w.rope_theta),
@@ -630,36 +638,31 @@ def run_e2e(eng, w, args, world, unit):
     import torch
     if w.name == "encode":
         return None  # the offline encode's input is the resident corpus; no per-step host input
-    L = eng.L
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype).pin_memory()  # noqa: E731
-    h_qr = [pin(t) for t in eng.qr_d]
-    h_q = [pin(t) for t in eng.q_d]
-    for src, dst in ((eng.qr_d, h_qr), (eng.q_d, h_q)):
-        for s, d_ in zip(src, dst):
-            d_.copy_(s)
-    # the decoded token's new local K/V row (one per sequence): last local slot
-    last = eng.loc_off[1:] - 1
-    idx = torch.from_numpy(last.astype(np.int64)).cuda()
-    h_k = [pin(t[idx]) for t in eng.kl_d]
-    h_v = [pin(t[idx]) for t in eng.vl_d]
-    for l in range(L):
-        h_k[l].copy_(eng.kl_d[l][idx])
-        h_v[l].copy_(eng.vl_d[l][idx])
-    h_out = [pin(t) for t in eng.out]
-    h_ids = [pin(t) for t in eng.ids]
-    h2d = sum(t.numel() * t.element_size() for lst in (h_qr, h_q, h_k, h_v) for t in lst)
-    d2h = sum(t.numel() * t.element_size() for lst in (h_out, h_ids) for t in lst)
+    # per step: every layer's query routing rows and attention queries, and the
+    # decoded token's new local K/V row of every sequence; back: outputs and ids
+    h_qr, h_q = pin(eng.qr_all), pin(eng.q_all)
+    h_qr.copy_(eng.qr_all)
+    h_q.copy_(eng.q_all)
+    idx = torch.from_numpy((eng.loc_off[1:] - 1).astype(np.int64)).cuda()  # last local slot of each sequence
+    h_k, h_v = pin(eng.kl_all[:, idx]), pin(eng.vl_all[:, idx])
+    h_k.copy_(eng.kl_all[:, idx])
+    h_v.copy_(eng.vl_all[:, idx])
+    d_k, d_v = torch.empty_like(eng.kl_all[:, idx]), torch.empty_like(eng.vl_all[:, idx])
+    h_out, h_ids = pin(eng.out_all), pin(eng.ids_all)
+    h2d = sum(t.numel() * t.element_size() for t in (h_qr, h_q, h_k, h_v))
+    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_ids))
 
     def step():
-        for l in range(L):
-            eng.qr_d[l].copy_(h_qr[l], non_blocking=True)
-            eng.q_d[l].copy_(h_q[l], non_blocking=True)
-            eng.kl_d[l][idx] = h_k[l].cuda(non_blocking=True)
-            eng.vl_d[l][idx] = h_v[l].cuda(non_blocking=True)
+        eng.qr_all.copy_(h_qr, non_blocking=True)
+        eng.q_all.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        eng.kl_all[:, idx] = d_k
+        eng.vl_all[:, idx] = d_v
         eng.run_step()
-        for l in range(L):
-            h_out[l].copy_(eng.out[l], non_blocking=True)
-            h_ids[l].copy_(eng.ids[l], non_blocking=True)
+        h_out.copy_(eng.out_all, non_blocking=True)
+        h_ids.copy_(eng.ids_all, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         step()
