@@ -83,6 +83,13 @@ def _load():
         lib.orc_attend.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P,
                                    f64, f64, f64, P, P]
         lib.orc_attend.restype = i32
+        lib.orc_route_f64.argtypes = [P, P, i64, i32, i32, P, P, i32, f64, i32, P, P, P]
+        lib.orc_route_f64.restype = i32
+        lib.orc_route_backward.argtypes = [P, P, i64, i32, i32, P, P, i32, f64, P, P, P, i32, P, P, P, P]
+        lib.orc_route_backward.restype = i32
+        lib.orc_attend_f64.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, f64, f64, f64, P, P,
+                                       P, P, P, P, P, P]
+        lib.orc_attend_f64.restype = i32
         _lib = lib
     return _lib
 
@@ -220,3 +227,86 @@ def attend(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, 
     if rc != 0:
         raise ValueError(f"orc_attend failed ({rc})")
     return out, lse
+
+
+# ------------------------------------------------- fp64 inputs and gradients
+
+def _f64(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    return bf16_to_f64(a) if a.dtype == np.uint16 else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def route_scores_f64(kbar_r, doc_chunk_off, qr, q_seq_off, eps=1e-8):
+    """Document scores [S, D] from fp64 inputs (same arithmetic as ``route``)."""
+    kr, q = _f64(kbar_r), _f64(qr)
+    dco = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
+    qso = np.ascontiguousarray(q_seq_off, dtype=np.int32)
+    n_docs, n_seq = dco.size - 1, qso.size - 1
+    ds = np.empty((n_seq, n_docs), np.float64)
+    ids = np.empty((n_seq, 1), np.int32)
+    sc = np.empty((n_seq, 1), np.float64)
+    rc = _load().orc_route_f64(_p(kr), _p(dco), n_docs, q.shape[1], q.shape[2], _p(q), _p(qso), n_seq, float(eps),
+                               1, _p(ds), _p(ids), _p(sc))
+    if rc != 0:
+        raise ValueError(f"orc_route_f64 failed ({rc})")
+    return ds
+
+
+def route_backward(kbar_r, doc_chunk_off, qr, q_seq_off, pair_seq, pair_doc, pair_dscore, eps=1e-8):
+    """Gradients of sum_p dscore_p * score(seq_p, doc_p): (dqr [T, hr, d],
+    dkr [P, hr, d], argmax_chunk [P], argmax_row [P])."""
+    kr, q = _f64(kbar_r), _f64(qr)
+    dco = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
+    qso = np.ascontiguousarray(q_seq_off, dtype=np.int32)
+    ps = np.ascontiguousarray(pair_seq, dtype=np.int32)
+    pd = np.ascontiguousarray(pair_doc, dtype=np.int32)
+    pg = np.ascontiguousarray(pair_dscore, dtype=np.float64)
+    T, hr, d = q.shape
+    dq = np.zeros((T, hr, d))
+    dk = np.empty((ps.size, hr, d))
+    ac = np.empty(ps.size, np.int64)
+    ar = np.empty(ps.size, np.int32)
+    rc = _load().orc_route_backward(_p(kr), _p(dco), dco.size - 1, hr, d, _p(q), _p(qso), qso.size - 1, float(eps),
+                                    _p(ps), _p(pd), _p(pg), ps.size, _p(dq), _p(dk), _p(ac), _p(ar))
+    if rc != 0:
+        raise ValueError(f"orc_route_backward failed ({rc})")
+    return dq, dk, ac, ar
+
+
+def attend_f64(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk, pos_offset,
+               rope_theta=1e6, scale=None, dout=None):
+    """Attention from fp64 inputs; with ``dout`` also the gradients. Returns
+    (out, lse) or (out, lse, dq, dk_loc, dv_loc, dmem_k, dmem_v)."""
+    q, kl, vl, mk, mv = (_f64(x) for x in (q, k_loc, v_loc, mem_k, mem_v))
+    qso = np.ascontiguousarray(q_seq_off, dtype=np.int32)
+    qst = np.ascontiguousarray(q_start, dtype=np.int32)
+    lo = np.ascontiguousarray(loc_off, dtype=np.int32)
+    so = np.ascontiguousarray(sel_off, dtype=np.int64)
+    sc = np.ascontiguousarray(sel_chunk, dtype=np.int64)
+    if sc.size == 0:
+        sc = np.zeros(1, np.int64)
+    n_q, hq, d = q.shape
+    hkv = kl.shape[1] if kl.size else mk.shape[1]
+    if kl.size == 0:
+        kl = np.zeros((1, hkv, d))
+        vl = np.zeros((1, hkv, d))
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((n_q, hq, d))
+    lse = np.empty((n_q, hq))
+    grads = None
+    if dout is not None:
+        go = np.ascontiguousarray(dout, dtype=np.float64)
+        n_sel = int(so[-1])
+        grads = [np.zeros((n_q, hq, d)), np.zeros(kl.shape), np.zeros(vl.shape),
+                 np.zeros((max(n_sel, 1), hkv, d)), np.zeros((max(n_sel, 1), hkv, d))]
+    rc = _load().orc_attend_f64(_p(q), _p(qso), _p(qst), qso.size - 1, hq, hkv, d, _p(kl), _p(vl), _p(lo), _p(mk),
+                                _p(mv), _p(so), _p(sc), float(pos_offset), float(rope_theta), float(scale), _p(out),
+                                _p(lse), _p(go) if grads else None, *([_p(g) for g in grads] if grads else [None] * 5))
+    if rc != 0:
+        raise ValueError(f"orc_attend_f64 failed ({rc})")
+    if grads is None:
+        return out, lse
+    n_sel = int(so[-1])
+    return (out, lse, grads[0], grads[1][: max(int(lo[-1]), 0)], grads[2][: max(int(lo[-1]), 0)],
+            grads[3][:n_sel], grads[4][:n_sel])

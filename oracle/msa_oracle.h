@@ -87,6 +87,29 @@ int orc_attend(const uint16_t* q, const int32_t* q_seq_off, const int32_t* q_sta
                double pos_offset, double rope_theta, double scale,
                double* out, double* lse);
 
+/* fp64-input twins of orc_route and orc_attend (same arithmetic; used for
+ * finite differences), and the gradients. orc_attend_f64 with dout != NULL
+ * computes dq [n_q, hq, d], dk_loc/dv_loc [n_loc, hkv, d] and dmem_k/dmem_v
+ * [n_sel, hkv, d] (selection order); the caller zeroes the accumulated ones.
+ * orc_route_backward: for (sequence, document, dL/dscore) triples, the
+ * gradient through the max's argmax (row, chunk) to dqr [n_rows, hr, d]
+ * (accumulated; caller zeroes) and dkr [n_pairs, hr, d]. */
+int orc_route_f64(const double* kbar_r, const int64_t* doc_chunk_off, int64_t n_docs,
+                  int hr, int d, const double* qr, const int32_t* q_seq_off, int n_seq,
+                  double eps, int top_k, double* doc_scores, int32_t* top_ids, double* top_scores);
+int orc_route_backward(const double* kbar_r, const int64_t* doc_chunk_off, int64_t n_docs, int hr, int d,
+                       const double* qr, const int32_t* q_seq_off, int n_seq, double eps,
+                       const int32_t* pair_seq, const int32_t* pair_doc, const double* pair_dscore, int n_pairs,
+                       double* dqr, double* dkr, int64_t* argmax_chunk, int32_t* argmax_row);
+int orc_attend_f64(const double* q, const int32_t* q_seq_off, const int32_t* q_start, int n_seq,
+                   int hq, int hkv, int d,
+                   const double* k_loc, const double* v_loc, const int32_t* loc_off,
+                   const double* mem_k, const double* mem_v,
+                   const int64_t* sel_off, const int64_t* sel_chunk,
+                   double pos_offset, double rope_theta, double scale,
+                   double* out, double* lse, const double* dout, double* dq, double* dk_loc, double* dv_loc,
+                   double* dmem_k, double* dmem_v);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_backward as grad_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "msa_oracle.c")
 
@@ -27,23 +28,32 @@ MUTANTS = {
     "encode_full_chunk_divisor": ("kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)n);",
                                   "kbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sk[i] / (double)chunk);"),
     "encode_norm_unrounded": ("double x = orc_bf16_to_double(b);", "double x = sr[(size_t)h * d + i] / (double)n + 1e-3;"),
-    "route_no_head_mean": ("double sc = cos_sum / (double)hr;", "double sc = cos_sum;"),
-    "route_mean_not_max": ("if (sc > best) best = sc;         /* max over rows and chunks */",
+    "route_no_head_mean": ("return cos_sum / (double)hr; /* mean over heads */", "return cos_sum;"),
+    "route_mean_not_max": ("if (sc > best) best = sc; /* max over rows and chunks */",
                            "best = (best == -INFINITY ? 0.0 : best) + sc;"),
-    "route_missing_knorm": ("cos_sum += dot * inv_q[(size_t)t * hr + h] * inv_k[(size_t)c * hr + h];",
-                            "cos_sum += dot * inv_q[(size_t)t * hr + h];"),
+    "route_missing_knorm": ("cos_sum += dot * inv_q[h] * inv_k[h];", "cos_sum += dot * inv_q[h];"),
     "route_ties_high_id": ("return (x->id > y->id) - (x->id < y->id);", "return (x->id < y->id) - (x->id > y->id);"),
-    "route_transposed_head": ("kbar_r + ((size_t)c * hr + h) * d, d);", "kbar_r + ((size_t)c * hr + (hr - 1 - h)) * d, d);"),
+    "route_transposed_head": ("kr, ((size_t)c * hr + h) * d, d);", "kr, ((size_t)c * hr + (hr - 1 - h)) * d, d);"),
     "attend_gqa_modulo": ("int kh = h / group;", "int kh = h % hkv;"),
-    "attend_causal_strict": ("for (int64_t j = 0; j < n_loc && j <= g; ++j) {", "for (int64_t j = 0; j < n_loc && j < g; ++j) {"),
-    "attend_no_query_offset": ("orc_rope(qv, d, pos_offset + (double)g, rope_theta);", "orc_rope(qv, d, (double)g, rope_theta);"),
+    "attend_causal_strict": ("for (int64_t j = 0; j < n_loc && j <= gq; ++j) {",
+                             "for (int64_t j = 0; j < n_loc && j < gq; ++j) {"),
+    "attend_no_query_offset": ("orc_rope(qv, d, pos_offset + (double)gq, rope_theta);",
+                               "orc_rope(qv, d, (double)gq, rope_theta);"),
+    "backward_no_softmax_term": ("double ds = p * (dp - D);", "double ds = p * dp;"),
+    "backward_q_not_rotated_back": ("orc_rope(g, d, -(pos_offset + (double)gq), rope_theta);", "(void)0;"),
+    "backward_local_k_not_rotated_back": ("orc_rope(kv, d, -(pos_offset + (double)gidx[j]), rope_theta);", "(void)0;"),
+    "backward_dv_unweighted": ("for (int i = 0; i < d; ++i) dv[i] += p * go[i];", "for (int i = 0; i < d; ++i) dv[i] += go[i];"),
+    "route_backward_no_norm_term": ("double gq = kv[i] * iq * ik - (nq > eps ? dot * ik * iq * iq * iq * qv[i] : 0.0);",
+                                    "double gq = kv[i] * iq * ik;"),
+    "route_backward_wrong_argmax": ("if (sc > best) { best = sc; cb = c; tb = t; }", "if (sc >= best) { best = sc; cb = c; tb = t; }"),
     "attend_lse_no_max": ("lse[(size_t)r * hq + h] = mx + log(den);", "lse[(size_t)r * hq + h] = log(den);"),
     "bf16_truncate": ("double r = nearbyint(ldexp(ax, -q));", "double r = floor(ldexp(ax, -q));"),
     "gather_skips_last_chunk": ("for (int64_t c = doc_chunk_off[doc]; c < doc_chunk_off[doc + 1]; ++c) {",
                                 "for (int64_t c = doc_chunk_off[doc]; c + 1 < doc_chunk_off[doc + 1]; ++c) {"),
 }
 
-PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+PIN_TESTS = ([getattr(pins, n) for n in dir(pins) if n.startswith("test_")] +
+             [getattr(grad_pins, n) for n in dir(grad_pins) if n.startswith("test_")])
 
 
 def _build(src_text, workdir, name):
