@@ -320,6 +320,43 @@ msa_status msa_attend_workspace(const msa_attend_args* args, size_t* bytes);
 msa_status msa_attend(const msa_attend_args* args, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* ------------------------------------------------------------------------
+ * Gradients (training). The pages present top-k routing plus sparse attention
+ * as one end-to-end differentiable operation trained with a generation loss
+ * and a contrastive routing loss ["MSA: Memory Sparse Attention", Abstract,
+ * Key Contributions; "MSA-arXiv26", 核心方法 (training)].
+ *
+ * msa_route_backward: for n_pairs (sequence, document, dL/dscore) triples
+ * (device arrays pair_seq, pair_doc, pair_dscore), the gradient of
+ * sum dscore * score(sequence, document). The score is a max over the
+ * sequence's rows and the document's chunks, so the gradient flows through its
+ * first argmax (row t*, chunk c*) in chunk-major, row-minor order:
+ *   d/dq_h = (k invq invk - [|q| > eps] (q.k) invk invq^3 q) / hr, symmetric in k.
+ * dqr [n_rows, hr, d] fp32 is ACCUMULATED (the caller zeroes it); dkr
+ * [n_pairs, hr, d] fp32 receives each triple's gradient for its argmax chunk,
+ * whose index goes to argmax_chunk [n_pairs] (-1 for a document without
+ * chunks) and whose row to argmax_row [n_pairs]. q_seq_off is HOST memory.
+ *
+ * msa_attend_backward: gradients of msa_attend for dout [n_q, hq, d] fp32.
+ * args is the forward's argument block with out_f32 and lse holding the
+ * forward's results (both required). Outputs (fp32, device): dq [n_q, hq, d]
+ * (w.r.t. the un-rotated queries), dk_loc and dv_loc [n_loc, hkv, d] (w.r.t.
+ * the un-rotated local keys and values; zero for local keys no row sees),
+ * dmem_k and dmem_v [sel_off[n_seq], hkv, d]: one row per selected memory
+ * row in selection order (a chunk selected by several sequences gets one row
+ * per selection; sum them to get the bank's gradient).
+ * ---------------------------------------------------------------------- */
+msa_status msa_route_backward(const msa_bank_layer* bank, const uint16_t* qr, const int32_t* q_seq_off,
+                              int32_t n_seq, int32_t n_rows, float eps, const int32_t* pair_seq,
+                              const int32_t* pair_doc, const float* pair_dscore, int32_t n_pairs,
+                              float* dqr, float* dkr, int64_t* argmax_chunk, int32_t* argmax_row,
+                              void* stream);
+
+msa_status msa_attend_backward_workspace(const msa_attend_args* args, size_t* bytes);
+msa_status msa_attend_backward(const msa_attend_args* args, const float* dout, float* dq, float* dk_loc,
+                               float* dv_loc, float* dmem_k, float* dmem_v, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Waits for `stream` and reports any pending CUDA error as MSA_ERR_CUDA. */
 msa_status msa_sync_check(void* stream);
 

@@ -94,10 +94,14 @@ _sig("msa_gather", [ctypes.POINTER(GatherArgsC), P])
 _sig("msa_attend_workspace", [ctypes.POINTER(AttendArgsC), ctypes.POINTER(ctypes.c_size_t)])
 _sig("msa_attend", [ctypes.POINTER(AttendArgsC), P, ctypes.c_size_t, P])
 _sig("msa_sync_check", [P])
+_sig("msa_route_backward", [ctypes.POINTER(BankLayerC), P, P, i32, i32, f32, P, P, P, i32, P, P, P, P, P])
+_sig("msa_attend_backward_workspace", [ctypes.POINTER(AttendArgsC), ctypes.POINTER(ctypes.c_size_t)])
+_sig("msa_attend_backward", [ctypes.POINTER(AttendArgsC), P, P, P, P, P, P, P, ctypes.c_size_t, P])
 
 EXPORTS = ["msa_status_string", "msa_last_error", "msa_version", "msa_encode_plan", "msa_encode",
            "msa_bank_norms", "msa_route_workspace", "msa_route", "msa_route_static", "msa_topk_merge", "msa_gather", "msa_attend_workspace",
-           "msa_attend", "msa_sync_check"]
+           "msa_attend", "msa_sync_check", "msa_route_backward", "msa_attend_backward_workspace",
+           "msa_attend_backward"]
 
 
 def _check(code: int, where: str) -> None:
@@ -295,6 +299,38 @@ def attend(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, 
                            max_sel, pos_offset, rope_theta, scale, out, out_f32, lse)
     _check(_lib.msa_attend(ctypes.byref(a), _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream)), "msa_attend")
+
+
+def route_backward(bank: BankLayer, qr, q_seq_off_host, pair_seq, pair_doc, pair_dscore, dqr, dkr, argmax_chunk,
+                   argmax_row, eps: float = 1e-8, stream=None) -> None:
+    """Gradient of sum dscore * score(seq, doc) over (seq, doc, dscore) triples
+    (device arrays). dqr [T, hr, 128] fp32 is accumulated (zero it first)."""
+    b = bank.c()
+    qso = _host_i32(q_seq_off_host)
+    _check(_lib.msa_route_backward(ctypes.byref(b), _ptr(qr), qso.ctypes.data, qso.size - 1, qr.shape[0], eps,
+                                   _ptr(pair_seq), _ptr(pair_doc), _ptr(pair_dscore), pair_seq.numel(), _ptr(dqr),
+                                   _ptr(dkr), _ptr(argmax_chunk), _ptr(argmax_row), _stream(stream)),
+           "msa_route_backward")
+
+
+def attend_backward_workspace(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
+                              max_sel, out_f32, lse, pos_offset=16.0, rope_theta=1e6, scale=0.0) -> int:
+    a, keep = _attend_args(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
+                           max_sel, pos_offset, rope_theta, scale, q, out_f32, lse)
+    n = ctypes.c_size_t()
+    _check(_lib.msa_attend_backward_workspace(ctypes.byref(a), ctypes.byref(n)), "msa_attend_backward_workspace")
+    return n.value
+
+
+def attend_backward(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk, max_sel,
+                    out_f32, lse, dout, dq, dk_loc, dv_loc, dmem_k, dmem_v, workspace, pos_offset=16.0,
+                    rope_theta=1e6, scale=0.0, stream=None) -> None:
+    """Gradients of ``attend`` given the forward's fp32 output and lse."""
+    a, keep = _attend_args(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
+                           max_sel, pos_offset, rope_theta, scale, q, out_f32, lse)
+    _check(_lib.msa_attend_backward(ctypes.byref(a), _ptr(dout), _ptr(dq), _ptr(dk_loc), _ptr(dv_loc), _ptr(dmem_k),
+                                    _ptr(dmem_v), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "msa_attend_backward")
 
 
 def sync_check(stream=None) -> None:

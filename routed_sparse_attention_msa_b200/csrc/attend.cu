@@ -26,6 +26,8 @@
 // The split count puts about two CTAs on every SM.
 #include <math.h>
 
+#include <algorithm>
+
 #include "msa_internal.cuh"
 
 namespace msa {
@@ -371,6 +373,351 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
   }
 }
 
+
+// ------------------------------------------------------------------ backward
+//
+// Gradients of the attention (the pages' end-to-end differentiable sparse
+// attention): with D = dout.out per (row, head), for every visible key j,
+//   p_j = exp(scale q'.k'_j - lse),  ds_j = p_j (dout.v_j - D),
+//   dq' = scale sum_j ds_j k'_j,  dk'_j = scale sum ds_j q',  dv_j = sum p_j dout,
+// primes are rotated vectors; dq and the local keys' gradients are rotated
+// back (by the negative angle), pooled memory keys are used as stored.
+
+// Rotation of the pair (x, y) of dimension i by minus the angle at `pos`.
+__device__ __forceinline__ void rotate_back(float& x, float& y, int i, double pos, double log2_theta) {
+  const double w = exp2(-2.0 * (double)i / (double)kHeadDim * log2_theta);
+  const double ang = pos * w;
+  const double two_pi = 6.283185307179586476925286766559;
+  const float r = (float)(ang - two_pi * rint(ang / two_pi));
+  float sn, cs;
+  sincosf(r, &sn, &cs);
+  const float a = x * cs + y * sn;
+  const float b = -x * sn + y * cs;
+  x = a;
+  y = b;
+}
+
+// D[row, head] = dout . out (one warp per (row, head)).
+__global__ void attend_bwd_prep_kernel(const __grid_constant__ AttnParams p, const float* __restrict__ dout,
+                                       float* __restrict__ Dvec) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (w >= (int64_t)p.n_q * p.hq) return;
+  const float4 a = reinterpret_cast<const float4*>(dout + w * kHeadDim)[lane];
+  const float4 b = reinterpret_cast<const float4*>(p.out_f32 + w * kHeadDim)[lane];
+  float x = a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  if (lane == 0) Dvec[w] = x;
+}
+
+// Stage rows of K (fp32, rotated for local keys) and V of keys [kb, kb+nb) of
+// sequence s into shared memory; `all_local` also stages local keys no row sees.
+template <int KB>
+__device__ __forceinline__ void stage_kv(const AttnParams& p, int s, int kvh, int64_t kb, int nb, int64_t n_mem,
+                                         int64_t mem_base, float (*Sk)[kPad], float (*Sv)[kPad]) {
+  const size_t row_stride = (size_t)p.hkv * kHeadDim;
+  for (int idx = threadIdx.x; idx < KB * (kHeadDim / 8); idx += kThreads) {
+    const int jj = idx >> 4, c8 = idx & 15;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a, va = a, vb = a;
+    if (jj < nb) {
+      const int64_t key = kb + jj;
+      uint4 vw;
+      if (key < n_mem) {
+        const int64_t r = p.sel_chunk ? p.sel_chunk[mem_base + key] : mem_base + key;
+        const size_t off = (size_t)r * row_stride + (size_t)kvh * kHeadDim + 8 * c8;
+        const uint4 kw = *reinterpret_cast<const uint4*>(p.mem_k + off);
+        vw = *reinterpret_cast<const uint4*>(p.mem_v + off);
+        a = make_float4(bf_lo(kw.x), bf_hi(kw.x), bf_lo(kw.y), bf_hi(kw.y));
+        b = make_float4(bf_lo(kw.z), bf_hi(kw.z), bf_lo(kw.w), bf_hi(kw.w));
+      } else {
+        const size_t lr = (size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh;
+        const float4* kp = reinterpret_cast<const float4*>(p.krot + lr * kHeadDim + 8 * c8);
+        a = kp[0];
+        b = kp[1];
+        vw = *reinterpret_cast<const uint4*>(p.v_loc + lr * kHeadDim + 8 * c8);
+      }
+      va = make_float4(bf_lo(vw.x), bf_hi(vw.x), bf_lo(vw.y), bf_hi(vw.y));
+      vb = make_float4(bf_lo(vw.z), bf_hi(vw.z), bf_lo(vw.w), bf_hi(vw.w));
+    }
+    *reinterpret_cast<float4*>(&Sk[jj][8 * c8]) = a;
+    *reinterpret_cast<float4*>(&Sk[jj][8 * c8 + 4]) = b;
+    *reinterpret_cast<float4*>(&Sv[jj][8 * c8]) = va;
+    *reinterpret_cast<float4*>(&Sv[jj][8 * c8 + 4]) = vb;
+  }
+}
+
+template <int VEC>
+struct BwdQSmem {
+  float q[VEC][kHeadDim];
+  float go[VEC][kHeadDim];
+  float k[kKeyBlock][kPad];
+  float v[kKeyBlock][kPad];
+  float ds[VEC][kKeyBlock];
+  float lse[VEC], D[VEC];
+  int g[VEC];
+};
+
+// dq: one CTA per (query tile, kv head), all keys of the sequence.
+template <int VEC>
+__global__ void __launch_bounds__(kThreads) attend_bwd_dq_kernel(const __grid_constant__ AttnParams p,
+                                                                 const float* __restrict__ dout,
+                                                                 const float* __restrict__ Dvec,
+                                                                 float* __restrict__ dq) {
+  constexpr int VH = VEC / 2, VW = VEC / 4;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BwdQSmem<VEC>& S = *reinterpret_cast<BwdQSmem<VEC>*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int kvh = blockIdx.y, tile = blockIdx.z;
+  const int s = seq_of(p.tile_off, p.n_seq, tile);
+  const int row0 = p.q_seq_off[s] + (tile - p.tile_off[s]) * p.rt;
+  const int nr = min(p.rt, p.q_seq_off[s + 1] - row0);
+  const int g0 = p.q_start[s] + (row0 - p.q_seq_off[s]);
+  const int64_t mem_base = p.sel_off[s];
+  const int64_t n_mem = p.sel_off[s + 1] - mem_base;
+  const int n_loc_s = p.loc_off[s + 1] - p.loc_off[s];
+  const int64_t n_keys = n_mem + max(0, min(n_loc_s, g0 + nr));
+
+  for (int idx = tid; idx < VEC * kHeadDim / 4; idx += kThreads) {
+    const int v = idx / (kHeadDim / 4), e4 = idx % (kHeadDim / 4);
+    const int rr = v / p.group, gg = v % p.group;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+    if (rr < nr) {
+      const size_t o = ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim;
+      x = reinterpret_cast<const float4*>(p.qrot + o)[e4];
+      y = reinterpret_cast<const float4*>(dout + o)[e4];
+    }
+    reinterpret_cast<float4*>(S.q[v])[e4] = x;
+    reinterpret_cast<float4*>(S.go[v])[e4] = y;
+  }
+  if (tid < VEC) {
+    const int rr = tid / p.group, gg = tid % p.group;
+    const size_t rh = (size_t)(row0 + rr) * p.hq + kvh * p.group + gg;
+    S.lse[tid] = rr < nr ? p.lse[rh] : 0.f;
+    S.D[tid] = rr < nr ? Dvec[rh] : 0.f;
+    S.g[tid] = rr < nr ? g0 + rr : -1;
+  }
+  float acc[VW][4];
+#pragma unroll
+  for (int i = 0; i < VW; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  const int d0 = 4 * lane;
+
+  for (int64_t kb = 0; kb < n_keys; kb += kKeyBlock) {
+    const int nb = (int)min((int64_t)kKeyBlock, n_keys - kb);
+    __syncthreads();
+    stage_kv<kKeyBlock>(p, s, kvh, kb, nb, n_mem, mem_base, S.k, S.v);
+    __syncthreads();
+    {  // ds for (vector, key): thread -> key jj, VH vectors
+      const int jj = tid & (kKeyBlock - 1);
+      const int vh = (tid >> 6) * VH;
+      float l[VH], dp[VH];
+#pragma unroll
+      for (int v = 0; v < VH; ++v) l[v] = dp[v] = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < kHeadDim / 4; ++c) {
+        const float4 kx = *reinterpret_cast<const float4*>(&S.k[jj][4 * c]);
+        const float4 vx = *reinterpret_cast<const float4*>(&S.v[jj][4 * c]);
+#pragma unroll
+        for (int v = 0; v < VH; ++v) {
+          const float4 qa = *reinterpret_cast<const float4*>(&S.q[vh + v][4 * c]);
+          const float4 ga = *reinterpret_cast<const float4*>(&S.go[vh + v][4 * c]);
+          l[v] += kx.x * qa.x + kx.y * qa.y + kx.z * qa.z + kx.w * qa.w;
+          dp[v] += vx.x * ga.x + vx.y * ga.y + vx.z * ga.z + vx.w * ga.w;
+        }
+      }
+      const int64_t key = kb + jj;
+      const int lj = key < n_mem ? -1 : (int)(key - n_mem);
+#pragma unroll
+      for (int v = 0; v < VH; ++v) {
+        const int g = S.g[vh + v];
+        const bool vis = jj < nb && g >= 0 && (lj < 0 || lj <= g);
+        const float pr = vis ? expf(l[v] * p.scale - S.lse[vh + v]) : 0.f;
+        S.ds[vh + v][jj] = pr * (dp[v] - S.D[vh + v]);
+      }
+    }
+    __syncthreads();
+    for (int j = 0; j < nb; ++j) {
+      const float4 x = *reinterpret_cast<const float4*>(&S.k[j][d0]);
+#pragma unroll
+      for (int i = 0; i < VW; ++i) {
+        const float w = S.ds[wid + 4 * i][j];
+        acc[i][0] += w * x.x;
+        acc[i][1] += w * x.y;
+        acc[i][2] += w * x.z;
+        acc[i][3] += w * x.w;
+      }
+    }
+  }
+  // rotate back and write: dims 4*lane..+3 pair with lane +- 16
+#pragma unroll
+  for (int i = 0; i < VW; ++i) {
+    const int v = wid + 4 * i;
+    const int rr = v / p.group, gg = v % p.group;
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mine = acc[i][e] * p.scale;
+      const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+      float x = lane < 16 ? mine : other, y = lane < 16 ? other : mine;  // (dim, dim + 64)
+      const int dim = 4 * (lane & 15) + e;
+      if (rr < nr) rotate_back(x, y, dim, p.pos_offset + (double)(g0 + rr), p.log2_theta);
+      o[e] = lane < 16 ? x : y;
+    }
+    if (rr < nr) {
+      const size_t base = ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim + d0;
+      *reinterpret_cast<float4*>(dq + base) = make_float4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+constexpr int kBwdKeys = 32;   // keys per dk/dv CTA
+constexpr int kBwdVec = 16;    // query vectors per step of the dk/dv loop
+
+struct BwdKVSmem {
+  float k[kBwdKeys][kPad];
+  float v[kBwdKeys][kPad];
+  float q[kBwdVec][kHeadDim];
+  float go[kBwdVec][kHeadDim];
+  float p[kBwdVec][kBwdKeys];
+  float ds[kBwdVec][kBwdKeys];
+  float lse[kBwdVec], D[kBwdVec];
+  int g[kBwdVec];
+};
+
+// dk, dv: one CTA per (32-key block, kv head, sequence), all query vectors of
+// the sequence. Every key of the sequence (visible to some row or not) is
+// written once: memory rows in selection order, local rows rotated back.
+__global__ void __launch_bounds__(kThreads) attend_bwd_dkdv_kernel(const __grid_constant__ AttnParams p,
+                                                                   const float* __restrict__ dout,
+                                                                   const float* __restrict__ Dvec,
+                                                                   float* __restrict__ dk_loc,
+                                                                   float* __restrict__ dv_loc,
+                                                                   float* __restrict__ dmem_k,
+                                                                   float* __restrict__ dmem_v) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BwdKVSmem& S = *reinterpret_cast<BwdKVSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int kvh = blockIdx.y, s = blockIdx.z;
+  const int64_t mem_base = p.sel_off[s];
+  const int64_t n_mem = p.sel_off[s + 1] - mem_base;
+  const int n_loc_s = p.loc_off[s + 1] - p.loc_off[s];
+  const int64_t n_all = n_mem + n_loc_s;
+  const int64_t kb = (int64_t)blockIdx.x * kBwdKeys;
+  if (kb >= n_all) return;
+  const int nb = (int)min((int64_t)kBwdKeys, n_all - kb);
+  stage_kv<kBwdKeys>(p, s, kvh, kb, nb, n_mem, mem_base, S.k, S.v);
+
+  const int jk = tid >> 2;          // key of this thread in the accumulation
+  const int dsl = (tid & 3) * 32;   // its 32 dimensions
+  float ak[32], av[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) ak[e] = av[e] = 0.f;
+
+  const int r0 = p.q_seq_off[s], r1 = p.q_seq_off[s + 1];
+  const int rows_per_step = kBwdVec / p.group;
+  for (int rb = r0; rb < r1; rb += rows_per_step) {
+    const int nr = min(rows_per_step, r1 - rb);
+    __syncthreads();  // staging above / previous step's q, go, p, ds no longer in use
+    for (int idx = tid; idx < kBwdVec * kHeadDim / 4; idx += kThreads) {
+      const int v = idx / (kHeadDim / 4), e4 = idx % (kHeadDim / 4);
+      const int rr = v / p.group, gg = v % p.group;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+      if (rr < nr) {
+        const size_t o = ((size_t)(rb + rr) * p.hq + kvh * p.group + gg) * kHeadDim;
+        x = reinterpret_cast<const float4*>(p.qrot + o)[e4];
+        y = reinterpret_cast<const float4*>(dout + o)[e4];
+      }
+      reinterpret_cast<float4*>(S.q[v])[e4] = x;
+      reinterpret_cast<float4*>(S.go[v])[e4] = y;
+    }
+    if (tid < kBwdVec) {
+      const int rr = tid / p.group, gg = tid % p.group;
+      const size_t rh = (size_t)(rb + rr) * p.hq + kvh * p.group + gg;
+      S.lse[tid] = rr < nr ? p.lse[rh] : 0.f;
+      S.D[tid] = rr < nr ? Dvec[rh] : 0.f;
+      S.g[tid] = rr < nr ? p.q_start[s] + (rb + rr - r0) : -1;
+    }
+    __syncthreads();
+    {  // p and ds for (vector, key): thread -> key (tid & 31), 4 vectors
+      const int jj = tid & 31;
+      const int v0 = (tid >> 5) * 4;
+      float l[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int c = 0; c < kHeadDim / 4; ++c) {
+        const float4 kx = *reinterpret_cast<const float4*>(&S.k[jj][4 * c]);
+        const float4 vx = *reinterpret_cast<const float4*>(&S.v[jj][4 * c]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 qa = *reinterpret_cast<const float4*>(&S.q[v0 + v][4 * c]);
+          const float4 ga = *reinterpret_cast<const float4*>(&S.go[v0 + v][4 * c]);
+          l[v] += kx.x * qa.x + kx.y * qa.y + kx.z * qa.z + kx.w * qa.w;
+          dp[v] += vx.x * ga.x + vx.y * ga.y + vx.z * ga.z + vx.w * ga.w;
+        }
+      }
+      const int64_t key = kb + jj;
+      const int lj = key < n_mem ? -1 : (int)(key - n_mem);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int g = S.g[v0 + v];
+        const bool vis = jj < nb && g >= 0 && (lj < 0 || lj <= g);
+        const float pr = vis ? expf(l[v] * p.scale - S.lse[v0 + v]) : 0.f;
+        S.p[v0 + v][jj] = pr;
+        S.ds[v0 + v][jj] = pr * (dp[v] - S.D[v0 + v]);
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int v = 0; v < kBwdVec; ++v) {
+      const float w_ds = S.ds[v][jk] * p.scale, w_p = S.p[v][jk];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 qa = *reinterpret_cast<const float4*>(&S.q[v][dsl + e]);
+        const float4 ga = *reinterpret_cast<const float4*>(&S.go[v][dsl + e]);
+        ak[e] += w_ds * qa.x; ak[e + 1] += w_ds * qa.y; ak[e + 2] += w_ds * qa.z; ak[e + 3] += w_ds * qa.w;
+        av[e] += w_p * ga.x; av[e + 1] += w_p * ga.y; av[e + 2] += w_p * ga.z; av[e + 3] += w_p * ga.w;
+      }
+    }
+  }
+  // write: thread slices 0/2 and 1/3 of one key are the rotation pairs (d, d + 64);
+  // the shuffle runs on every lane, the rotation only for local keys
+  const int64_t key = kb + jk;
+  const bool local = key >= n_mem;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float other = __shfl_xor_sync(0xffffffffu, ak[e], 2);
+    if (local && jk < nb) {
+      float x = (tid & 2) ? other : ak[e], y = (tid & 2) ? ak[e] : other;
+      rotate_back(x, y, (dsl & 63) + e, p.pos_offset + (double)(key - n_mem), p.log2_theta);
+      ak[e] = (tid & 2) ? y : x;
+    }
+  }
+  if (jk >= nb) return;
+  float* dk;
+  float* dv;
+  if (!local) {
+    const size_t o = ((size_t)(mem_base + key) * p.hkv + kvh) * kHeadDim + dsl;
+    dk = dmem_k + o;
+    dv = dmem_v + o;
+  } else {
+    const size_t o = ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim + dsl;
+    dk = dk_loc + o;
+    dv = dv_loc + o;
+  }
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    *reinterpret_cast<float4*>(dk + e) = make_float4(ak[e], ak[e + 1], ak[e + 2], ak[e + 3]);
+    *reinterpret_cast<float4*>(dv + e) = make_float4(av[e], av[e + 1], av[e + 2], av[e + 3]);
+  }
+}
+
 struct Shape {
   int vec, rt, n_tiles, n_splits, n_loc;
 };
@@ -446,13 +793,11 @@ size_t attend_workspace(const msa_attend_args& a, int* n_splits_out) {
   return layout(a, sh).total;
 }
 
-msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
-  const Shape sh = plan(a);
-  const Layout L = layout(a, sh);
-  AttnParams P{};  // kernel parameter block (4.3 KB: large kernel parameters, CUDA >= 12.1)
+namespace {
+
+void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, char* w, AttnParams& P) {
   P.q = a.q; P.k_loc = a.k_loc; P.v_loc = a.v_loc; P.mem_k = a.mem_k; P.mem_v = a.mem_v;
   P.sel_off = a.sel_off; P.sel_chunk = a.sel_chunk;
-  char* w = reinterpret_cast<char*>(ws);
   P.qrot = reinterpret_cast<float*>(w + L.qrot);
   P.krot = reinterpret_cast<float*>(w + L.krot);
   P.part_o = reinterpret_cast<float*>(w + L.part_o);
@@ -475,13 +820,41 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   P.q_seq_off[a.n_seq] = a.q_seq_off[a.n_seq];
   P.loc_off[a.n_seq] = a.loc_off[a.n_seq];
   P.tile_off[a.n_seq] = t;
+}
 
+msa_status launch_rope(const AttnParams& P, const msa_attend_args& a, const Shape& sh, cudaStream_t st) {
   int64_t n = (int64_t)a.n_q * a.hq * 64 + (int64_t)sh.n_loc * a.hkv * 64;
   const int64_t nt = (int64_t)sh.n_tiles * a.hkv;
   if (n < nt) n = nt;
   cudaError_t e = launch_pdl(rope_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: rotate queries and local keys");
-  msa_status s = launch_check("attend: rotate queries and local keys");
+  return launch_check("attend: rotate queries and local keys");
+}
+
+template <int VEC>
+msa_status launch_bwd_dq(const AttnParams& P, const float* dout, const float* Dvec, float* dq, dim3 grid,
+                         cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attend_bwd_dq_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(BwdQSmem<VEC>));
+    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
+    attr = true;
+  }
+  cudaError_t e = launch_pdl(attend_bwd_dq_kernel<VEC>, grid, dim3(kThreads), sizeof(BwdQSmem<VEC>), st, P, dout,
+                             Dvec, dq);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: dq");
+  return launch_check("attend backward: dq");
+}
+
+}  // namespace
+
+msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
+  const Shape sh = plan(a);
+  const Layout L = layout(a, sh);
+  AttnParams P{};  // kernel parameter block (4.3 KB: large kernel parameters, CUDA >= 12.1)
+  fill_params(a, sh, L, reinterpret_cast<char*>(ws), P);
+  msa_status s = launch_rope(P, a, sh, st);
   if (s != MSA_OK) return s;
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
@@ -489,6 +862,53 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
     case 8: return launch_vec<8>(P, grid, st);
     default: return launch_vec<16>(P, grid, st);
   }
+}
+
+size_t attend_backward_workspace(const msa_attend_args& a) {
+  const Shape sh = plan(a);
+  const Layout L = layout(a, sh);
+  return L.total + align_up((size_t)a.n_q * a.hq * sizeof(float), 256);
+}
+
+msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, float* dq, float* dk_loc,
+                                  float* dv_loc, float* dmem_k, float* dmem_v, void* ws, cudaStream_t st) {
+  const Shape sh = plan(a);
+  const Layout L = layout(a, sh);
+  AttnParams P{};
+  char* w = reinterpret_cast<char*>(ws);
+  fill_params(a, sh, L, w, P);
+  float* Dvec = reinterpret_cast<float*>(w + L.total);
+  msa_status s = launch_rope(P, a, sh, st);
+  if (s != MSA_OK) return s;
+  const int64_t warps = (int64_t)a.n_q * a.hq;
+  cudaError_t e = launch_pdl(attend_bwd_prep_kernel, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, P,
+                             dout, Dvec);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: prep");
+  s = launch_check("attend backward: prep");
+  if (s != MSA_OK) return s;
+  dim3 gq(1, (unsigned)a.hkv, (unsigned)sh.n_tiles);
+  switch (sh.vec) {
+    case 4: s = launch_bwd_dq<4>(P, dout, Dvec, dq, gq, st); break;
+    case 8: s = launch_bwd_dq<8>(P, dout, Dvec, dq, gq, st); break;
+    default: s = launch_bwd_dq<16>(P, dout, Dvec, dq, gq, st); break;
+  }
+  if (s != MSA_OK) return s;
+  int max_loc = 0;
+  for (int q = 0; q < a.n_seq; ++q) max_loc = std::max(max_loc, a.loc_off[q + 1] - a.loc_off[q]);
+  const int64_t max_keys = a.max_sel + max_loc;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(attend_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(BwdKVSmem));
+    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
+    attr = true;
+  }
+  dim3 gk((unsigned)((max_keys + kBwdKeys - 1) / kBwdKeys > 0 ? (max_keys + kBwdKeys - 1) / kBwdKeys : 1),
+          (unsigned)a.hkv, (unsigned)a.n_seq);
+  e = launch_pdl(attend_bwd_dkdv_kernel, gk, dim3(kThreads), sizeof(BwdKVSmem), st, P, dout, Dvec, dk_loc, dv_loc,
+                 dmem_k, dmem_v);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: dk, dv");
+  return launch_check("attend backward: dk, dv");
 }
 
 }  // namespace msa

@@ -370,6 +370,48 @@ msa_status msa_attend(const msa_attend_args* a, void* ws, size_t ws_bytes, void*
   return launch_attend(*a, ws, (cudaStream_t)stream);
 }
 
+// ---------------------------------------------------------------- backward
+
+msa_status msa_route_backward(const msa_bank_layer* b, const uint16_t* qr, const int32_t* q_seq_off, int32_t n_seq,
+                              int32_t n_rows, float eps, const int32_t* pair_seq, const int32_t* pair_doc,
+                              const float* pair_dscore, int32_t n_pairs, float* dqr, float* dkr,
+                              int64_t* argmax_chunk, int32_t* argmax_row, void* stream) {
+  msa_status s = check_bank(b, false);
+  if (s != MSA_OK) return s;
+  if (n_seq <= 0 || n_seq > kMaxSeq || n_pairs < 0) return fail(MSA_ERR_INVALID_ARG, "route_backward: bad sizes");
+  if (!(eps > 0.f)) return fail(MSA_ERR_INVALID_ARG, "route_backward: eps must be > 0");
+  if (!q_seq_off || q_seq_off[0] != 0 || q_seq_off[n_seq] != n_rows)
+    return fail(MSA_ERR_INVALID_ARG, "route_backward: q_seq_off must start at 0 and end at n_rows");
+  for (int i = 0; i < n_seq; ++i)
+    if (q_seq_off[i + 1] <= q_seq_off[i]) return fail(MSA_ERR_INVALID_ARG, "route_backward: sequence %d has no rows", i);
+  if (n_pairs > 0 && (!qr || !pair_seq || !pair_doc || !pair_dscore || !dqr || !dkr || !argmax_chunk || !argmax_row))
+    return fail(MSA_ERR_INVALID_ARG, "route_backward: NULL pointer");
+  return launch_route_backward(*b, qr, q_seq_off, n_seq, eps, pair_seq, pair_doc, pair_dscore, n_pairs, dqr, dkr,
+                               argmax_chunk, argmax_row, (cudaStream_t)stream);
+}
+
+msa_status msa_attend_backward_workspace(const msa_attend_args* a, size_t* bytes) {
+  msa_status s = check_attend(a);
+  if (s != MSA_OK) return s;
+  if (!bytes) return fail(MSA_ERR_INVALID_ARG, "attend_backward_workspace: bytes is NULL");
+  *bytes = attend_backward_workspace(*a);
+  return MSA_OK;
+}
+
+msa_status msa_attend_backward(const msa_attend_args* a, const float* dout, float* dq, float* dk_loc, float* dv_loc,
+                               float* dmem_k, float* dmem_v, void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_attend(a);
+  if (s != MSA_OK) return s;
+  if (!a->out_f32 || !a->lse) return fail(MSA_ERR_INVALID_ARG, "attend_backward: the forward's out_f32 and lse are required");
+  if (!dout || !dq) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dout or dq");
+  if (a->loc_off[a->n_seq] > 0 && (!dk_loc || !dv_loc)) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dk_loc/dv_loc");
+  if (a->max_sel > 0 && (!dmem_k || !dmem_v)) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dmem_k/dmem_v");
+  const size_t need = attend_backward_workspace(*a);
+  if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "attend_backward: workspace %zu B, need %zu B", ws_bytes, need);
+  if (a->n_q == 0) return MSA_OK;
+  return launch_attend_backward(*a, dout, dq, dk_loc, dv_loc, dmem_k, dmem_v, ws, (cudaStream_t)stream);
+}
+
 msa_status msa_sync_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaGetLastError();

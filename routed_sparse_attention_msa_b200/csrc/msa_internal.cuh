@@ -113,6 +113,12 @@ bool score_tc_supported(const RoutePlan& p);
 bool score_tc_built();
 int tc_error_take();  // 1 if a tensor-core kernel's bounded wait ran out since the last call
 
+// route_backward.cu
+msa_status launch_route_backward(const msa_bank_layer& b, const uint16_t* qr, const int32_t* q_seq_off, int n_seq,
+                                 float eps, const int32_t* pair_seq, const int32_t* pair_doc,
+                                 const float* pair_dscore, int n_pairs, float* dqr, float* dkr,
+                                 int64_t* argmax_chunk, int32_t* argmax_row, cudaStream_t st);
+
 // topk.cu
 size_t topk_workspace(int n_seq, int64_t n_docs, int k);
 msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k,
@@ -132,5 +138,8 @@ msa_status launch_gather_pull(const msa_bank_layer& b, const int64_t* sel_off,
 // attend.cu
 size_t attend_workspace(const msa_attend_args& a, int* n_splits_out);
 msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st);
+size_t attend_backward_workspace(const msa_attend_args& a);
+msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, float* dq, float* dk_loc,
+                                  float* dv_loc, float* dmem_k, float* dmem_v, void* ws, cudaStream_t st);
 
 }  // namespace msa
