@@ -50,6 +50,13 @@ def parse_args():
                         "if host RAM allows)")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count (0: as defined)")
     p.add_argument("--seqs", type=int, default=0, help="override the workload's sequence count (0: as defined)")
+    p.add_argument("--mode", choices=["decode", "train", "sharded", "interleave"], default="decode",
+                   help="decode: the routed decode step (default); train: decode step plus the gradients of "
+                        "attention and of the routing scores; sharded: routing of every layer split into "
+                        "--shards document shards merged by the top-k merge (Memory Parallel, emulated on one "
+                        "GPU); interleave: --hops routing hops per layer (Memory Interleave)")
+    p.add_argument("--shards", type=int, default=8)
+    p.add_argument("--hops", type=int, default=3)
     p.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
                    help="replay each step as one CUDA graph (auto: on unless the copy-engine gather needs host syncs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -279,7 +286,52 @@ class Routed:
         self.ws_attend = torch.empty(msa.attend_workspace(*a0, pos_offset=self.pos_offset, rope_theta=w.rope_theta),
                                      dtype=torch.uint8, device="cuda")
         self.mode = msa.GATHER_DEVICE_PULL if args.gather == "pull" else msa.GATHER_COPY_ENGINE
+        self.run_mode = args.mode
+        if args.mode == "interleave" and S != 1:
+            raise SystemExit("--mode interleave follows one sequence; use a workload with one sequence")
+        if args.mode == "train":
+            self._setup_train(a0)
+        elif args.mode == "sharded":
+            self._setup_sharded(args.shards)
         torch.cuda.synchronize()
+
+    def _setup_train(self, a0):
+        """Buffers for the gradients: forward fp32 output and lse, dL/dout, and
+        dL/dscore for every routed (sequence, document)."""
+        torch, msa, w = self.torch, self.msa, self.w
+        S, kk, d = self.S, self.kk, w.d
+        self.out_f32 = torch.empty((self.L, self.Tq, w.hq, d), dtype=torch.float32, device="cuda")
+        self.lse = torch.empty((self.L, self.Tq, w.hq), dtype=torch.float32, device="cuda")
+        self.dout = torch.from_numpy(synth.bits_to_f64(synth.normal_bf16_host(
+            self.Tq * w.hq * d, synth.tid("q_att", 99))).astype(np.float32).reshape(self.Tq, w.hq, d)).cuda()
+        self.dq = torch.empty((self.Tq, w.hq, d), dtype=torch.float32, device="cuda")
+        self.dkl = torch.empty((S * self.Lloc, w.hkv, d), dtype=torch.float32, device="cuda")
+        self.dvl = torch.empty_like(self.dkl)
+        self.dmk = torch.empty((self.cap, w.hkv, d), dtype=torch.float32, device="cuda")
+        self.dmv = torch.empty_like(self.dmk)
+        self.pair_seq = torch.arange(S, dtype=torch.int32, device="cuda").repeat_interleave(kk)
+        self.pair_dscore = torch.linspace(-1.0, 1.0, S * kk, device="cuda")
+        self.dqr = torch.empty((self.T, w.hr, d), dtype=torch.float32, device="cuda")
+        self.dkr = torch.empty((S * kk, w.hr, d), dtype=torch.float32, device="cuda")
+        self.argc = torch.empty(S * kk, dtype=torch.int64, device="cuda")
+        self.argr = torch.empty(S * kk, dtype=torch.int32, device="cuda")
+        self.ws_bwd = torch.empty(msa.attend_backward_workspace(*a0, self.out_f32[0], self.lse[0],
+                                                                pos_offset=self.pos_offset,
+                                                                rope_theta=w.rope_theta),
+                                  dtype=torch.uint8, device="cuda")
+
+    def _setup_sharded(self, n_shards):
+        from routed_sparse_attention_msa_b200 import memory_parallel as mp
+        torch, msa = self.torch, self.msa
+        self.shard_ranges = mp.shard_ranges(self.dco, n_shards)
+        self.shards = [[mp.make_shard(self.banks[l], self.dco, d0, d1) for d0, d1 in self.shard_ranges]
+                       for l in range(self.L)]
+        self.shard_ids = torch.empty((n_shards, self.S, self.k), dtype=torch.int32, device="cuda")
+        self.shard_sc = torch.empty((n_shards, self.S, self.k), dtype=torch.float32, device="cuda")
+        self.shard_ws = [torch.empty(max(msa.route_workspace(sh.layer, self.S, self.T, self.k), 256),
+                                     dtype=torch.uint8, device="cuda") if sh.n_docs else None
+                         for sh in self.shards[0]]
+        self.mp = mp
 
     def _host_content_layers(self) -> int:
         need = 2 * self.C * self.w.hkv * self.w.d * 2 * self.L
@@ -299,18 +351,48 @@ class Routed:
 
     def layer(self, l, ev=None):
         msa = self.msa
-        if ev is not None:
-            msa.score_events(ev[0], ev[1])
-        msa.route(self.banks[l], self.qr_d[l], self.qso, self.k, self.ids[l], self.scores[l], self.ws_route,
-                  eps=self.w.eps)
+        if self.run_mode == "sharded":
+            # Memory Parallel, one shard after another: route every shard, merge
+            for g, sh in enumerate(self.shards[l]):
+                if g == 0 and ev is not None:
+                    msa.score_events(ev[0], ev[1])
+                if sh.n_docs == 0:
+                    self.shard_ids[g].fill_(-1)
+                    continue
+                self.mp.route_local(sh, self.qr_d[l], self.qso, self.k, self.shard_ids[g], self.shard_sc[g],
+                                    self.shard_ws[g], eps=self.w.eps)
+            msa.topk_merge(self.shard_ids, self.shard_sc, [d0 for d0, _ in self.shard_ranges], self.kk,
+                           self.ids[l], self.scores[l])
+        elif self.run_mode == "interleave":
+            from routed_sparse_attention_msa_b200.interleave import memory_interleave
+            if ev is not None:
+                msa.score_events(ev[0], ev[1])
+            fetched, per_hop, _ = memory_interleave(self.banks[l], self.dco, self.qr_d[l], self.k, self.args.hops,
+                                                    eps=self.w.eps)
+            self.ids[l].copy_(self.torch.from_numpy(per_hop[-1][None]).to(self.ids[l].device))
+        else:
+            if ev is not None:
+                msa.score_events(ev[0], ev[1])
+            msa.route(self.banks[l], self.qr_d[l], self.qso, self.k, self.ids[l], self.scores[l], self.ws_route,
+                      eps=self.w.eps)
         if self.on_host:
             msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel, self.stage_k, self.stage_v,
                        mode=self.mode, doc_chunk_off_host=self.dco, top_ids_host=self.ids_host,
                        copy_stream=self.copy_stream, done_event=self.copy_done)
         else:
             msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel)
-        msa.attend(*self._attend_args(l), self.out[l], self.ws_attend, pos_offset=self.pos_offset,
-                   rope_theta=self.w.rope_theta)
+        if self.run_mode != "train":
+            msa.attend(*self._attend_args(l), self.out[l], self.ws_attend, pos_offset=self.pos_offset,
+                       rope_theta=self.w.rope_theta)
+            return
+        a = self._attend_args(l)
+        msa.attend(*a, self.out[l], self.ws_attend, out_f32=self.out_f32[l], lse=self.lse[l],
+                   pos_offset=self.pos_offset, rope_theta=self.w.rope_theta)
+        msa.attend_backward(*a, self.out_f32[l], self.lse[l], self.dout, self.dq, self.dkl, self.dvl, self.dmk,
+                            self.dmv, self.ws_bwd, pos_offset=self.pos_offset, rope_theta=self.w.rope_theta)
+        self.dqr.zero_()
+        msa.route_backward(self.banks[l], self.qr_d[l], self.qso, self.pair_seq, self.ids[l].view(-1),
+                           self.pair_dscore, self.dqr, self.dkr, self.argc, self.argr, eps=self.w.eps)
 
     def step(self, evs=None):
         for l in range(self.L):
@@ -321,7 +403,11 @@ class Routed:
 
     def score_bytes_per_launch(self) -> float:
         w = self.w
-        return self.C * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+        C = self.C
+        if self.run_mode == "sharded":  # the timed launch is shard 0's
+            d0, d1 = self.shard_ranges[0]
+            C = int(self.dco[d1] - self.dco[d0])
+        return C * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
 
     def check_planted(self):
         """Every layer's routed set must be its planted set (a property of the inputs)."""
@@ -523,12 +609,12 @@ def run_ours(args):
         return 0
 
     planted_ok = None
-    if w.name != "encode":
+    if w.name != "encode" and args.mode != "interleave":
         bad = eng.check_planted()
         planted_ok = bad == 0
 
     # ---- timed region: K steps, inputs resident in HBM
-    use_graph = args.graph == "on" or (args.graph == "auto" and not (
+    use_graph = args.graph == "on" or (args.graph == "auto" and args.mode != "interleave" and not (
         w.name != "encode" and w.content_on_host and args.gather == "copy"))
     graph = None
     if use_graph:
@@ -614,7 +700,11 @@ def run_ours(args):
                    "sample": (f"one routing layer ({r['chunks']} chunks, {r['tokens']} memory tokens x sequences): "
                               f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
 
-    extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None}
+    extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None, "mode": args.mode}
+    if args.mode == "sharded":
+        extra["shards"] = args.shards
+    if args.mode == "interleave":
+        extra["hops"] = args.hops
     if planted_ok is not None:
         extra["planted_sets_retrieved"] = planted_ok
     if w.name != "encode" and w.content_on_host:
