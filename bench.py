@@ -42,7 +42,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
-    p.add_argument("--score-kernel", choices=["auto", "simt", "tc"], default="auto")
+    p.add_argument("--score-kernel", choices=["auto", "simt", "tc", "tc_rows"], default="auto")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
     p.add_argument("--content-layers", type=int, default=1,
@@ -55,6 +55,9 @@ def parse_args():
                         "attention and of the routing scores; sharded: routing of every layer split into "
                         "--shards document shards merged by the top-k merge (Memory Parallel, emulated on one "
                         "GPU); interleave: --hops routing hops per layer (Memory Interleave)")
+    p.add_argument("--prefill", action="store_true",
+                   help="time the prefill step instead: every sequence routes and attends with its prefill rows "
+                        "(1m: 128, 10m: 64 per sequence), causal over those rows")
     p.add_argument("--shards", type=int, default=8)
     p.add_argument("--hops", type=int, default=3)
     p.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
@@ -589,6 +592,10 @@ def run_ours(args):
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs
+    if args.prefill:
+        if not w.prefill_rows:
+            raise SystemExit(f"workload {w.name} has no prefill rows")
+        w.route_rows = w.attn_rows = w.loc_len = w.prefill_rows
     metric, unit = metric_of(w.name)
     eng = Encode(w, args, local) if w.name == "encode" else Routed(w, args, local)
     L = eng.L
@@ -705,6 +712,8 @@ def run_ours(args):
         extra["shards"] = args.shards
     if args.mode == "interleave":
         extra["hops"] = args.hops
+    if args.prefill:
+        extra["step"] = "prefill"
     if planted_ok is not None:
         extra["planted_sets_retrieved"] = planted_ok
     if w.name != "encode" and w.content_on_host:

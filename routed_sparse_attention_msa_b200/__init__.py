@@ -149,8 +149,10 @@ def score_events(begin, end) -> None:
 
 
 def set_score_kernel(which: str) -> str:
-    """'auto', 'simt' (CUDA cores) or 'tc' (tensor cores); returns the previous setting."""
-    names = ["auto", "simt", "tc"]
+    """'auto', 'simt' (CUDA cores), 'tc' (tensor cores, per-head accumulators)
+    or 'tc_rows' (tensor cores, folded scales, for many query rows); returns
+    the previous setting."""
+    names = ["auto", "simt", "tc", "tc_rows"]
     return names[_lib.msa_debug_set_score_kernel(names.index(which))]
 
 

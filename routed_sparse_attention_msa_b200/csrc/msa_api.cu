@@ -14,7 +14,8 @@ namespace msa {
 
 namespace {
 thread_local char g_err[512] = "";
-int g_score_kernel = 0;  // 0 auto, 1 CUDA cores, 2 tensor cores
+int g_score_kernel = 0;  // 0 auto, 1 CUDA cores, 2 tensor cores, 3 tensor cores (many rows)
+constexpr int kManyRows = 64;  // above this many query rows the many-row scorer is chosen
 thread_local cudaEvent_t g_score_ev[2] = {nullptr, nullptr};
 }  // namespace
 
@@ -70,14 +71,18 @@ msa_status check_bank(const msa_bank_layer* b, bool need_content) {
 }
 
 struct RouteLayout {
-  size_t invq, doc_key, topk, total;
+  size_t invq, qhat, doc_key, topk, total;
 };
 
+// Workspace of one route call: query scales, the scaled query rows of the
+// many-row scorer (eight routing heads only), document keys, top-k state.
 RouteLayout route_layout(const msa_bank_layer* b, int n_seq, int n_rows, int top_k) {
   RouteLayout L;
   int k = top_k < b->n_docs ? top_k : (int)b->n_docs;
   L.invq = 0;
-  L.doc_key = align_up((size_t)n_rows * b->hr * sizeof(float), 256);
+  L.qhat = align_up((size_t)n_rows * b->hr * sizeof(float), 256);
+  const size_t qhat_bytes = b->hr == 8 ? (size_t)n_rows * b->hr * b->d * sizeof(uint16_t) : 0;
+  L.doc_key = L.qhat + align_up(qhat_bytes, 256);
   L.topk = L.doc_key + align_up((size_t)n_seq * b->n_docs * sizeof(uint32_t), 256);
   L.total = L.topk + topk_workspace(n_seq, b->n_docs, k);
   return L;
@@ -112,11 +117,12 @@ const char* msa_last_error(void) { return g_err; }
 int msa_version(void) { return MSA_VERSION; }
 
 // Selects the routing score kernel for later msa_route calls in this process:
-// 0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core kernel. A testing and
+// 0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core kernel (per-head
+// accumulators), 3 = tensor-core kernel for many rows. A testing and
 // benchmarking control; not declared in msa.h.
 int msa_debug_set_score_kernel(int which) {
   int old = g_score_kernel;
-  if (which >= 0 && which <= 2) g_score_kernel = which;
+  if (which >= 0 && which <= 3) g_score_kernel = which;
   return old;
 }
 
@@ -224,16 +230,22 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   p.n_chunks = b->n_chunks; p.n_docs = b->n_docs; p.hr = b->hr; p.n_rows = n_rows; p.n_seq = n_seq;
   for (int i = 0; i <= n_seq; ++i) p.q_seq_off[i] = q_seq_off[i];
   p.invq = reinterpret_cast<float*>(w + L.invq);
+  p.qhat = L.doc_key > L.qhat ? reinterpret_cast<uint16_t*>(w + L.qhat) : nullptr;
   p.doc_key = reinterpret_cast<uint32_t*>(w + L.doc_key);
   p.zero = w + L.doc_key;
   p.zero_bytes = L.total - L.doc_key;  // a multiple of 256
   s = launch_qprep(p, eps, st);
   if (s != MSA_OK) return s;
   if (b->n_chunks > 0) {
-    bool tc = g_score_kernel == 2 || (g_score_kernel == 0 && score_tc_supported(p));
-    if (tc && !score_tc_supported(p)) return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
+    // automatic: many rows -> the folded-scale contraction, a few -> per-head
+    // tensor-core accumulators, other head counts -> CUDA cores
+    int which = g_score_kernel;
+    if (which == 0)
+      which = score_pf_supported(p) && n_rows > kManyRows ? 3 : score_tc_supported(p) ? 2 : 1;
+    if ((which == 2 && !score_tc_supported(p)) || (which == 3 && !score_pf_supported(p)))
+      return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
     record_debug_event(0, st);
-    s = tc ? launch_score_tc(p, st) : launch_score_simt(p, st);
+    s = which == 3 ? launch_score_pf(p, st) : which == 2 ? launch_score_tc(p, st) : launch_score_simt(p, st);
     record_debug_event(1, st);
     if (s != MSA_OK) return s;
   }
@@ -416,7 +428,8 @@ msa_status msa_sync_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sync_check");
-  if (tc_error_take()) return fail(MSA_ERR_TIMEOUT, "sync_check: a tensor-core scoring kernel gave up on a wait");
+  const int e_tc = tc_error_take(), e_pf = pf_error_take();
+  if (e_tc || e_pf) return fail(MSA_ERR_TIMEOUT, "sync_check: a tensor-core scoring kernel gave up on a wait");
   return MSA_OK;
 }
 

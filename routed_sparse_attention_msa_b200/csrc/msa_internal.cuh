@@ -99,6 +99,7 @@ struct RoutePlan {
   int32_t hr, n_rows, n_seq;
   int32_t q_seq_off[kMaxSeq + 1];
   float* invq;                 // ws [T, hr]: 1 / (hr * max(||q||, eps))
+  uint16_t* qhat;              // ws [T, hr, d]: bf16(qr * invq) (hr = 8 only, else NULL)
   uint32_t* doc_key;           // ws [S, D]: ordered doc scores (0 = none)
   void* zero;                  // ws bytes to clear before scoring (doc keys, top-k state)
   size_t zero_bytes;           // multiple of 16
@@ -112,6 +113,10 @@ msa_status launch_score_tc(const RoutePlan& p, cudaStream_t st);
 bool score_tc_supported(const RoutePlan& p);
 bool score_tc_built();
 int tc_error_take();  // 1 if a tensor-core kernel's bounded wait ran out since the last call
+// score_pf.cu: the many-row (prefill) tensor-core scorer
+msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st);
+bool score_pf_supported(const RoutePlan& p);
+int pf_error_take();
 
 // route_backward.cu
 msa_status launch_route_backward(const msa_bank_layer& b, const uint16_t* qr, const int32_t* q_seq_off, int n_seq,

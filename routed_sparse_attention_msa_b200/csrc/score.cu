@@ -20,10 +20,13 @@
 namespace msa {
 namespace {
 
-// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)); the whole grid
-// also clears the scoring workspace (document keys and top-k state).
+// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)) and, when qhat
+// is given, the scaled row bf16(qr * invq) that the many-row scorer
+// contracts; the whole grid also clears the scoring workspace (document keys
+// and top-k state).
 __global__ void qprep_kernel(const uint16_t* __restrict__ qr, int n_rows, int hr, float eps,
-                             float* __restrict__ invq, uint4* __restrict__ zero, int64_t zero_vecs) {
+                             float* __restrict__ invq, uint16_t* __restrict__ qhat, uint4* __restrict__ zero,
+                             int64_t zero_vecs) {
   pdl_wait();
   pdl_trigger();
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -36,7 +39,11 @@ __global__ void qprep_kernel(const uint16_t* __restrict__ qr, int n_rows, int hr
   float ss = a * a + b * b + c * c + d * d;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) invq[w] = 1.0f / ((float)hr * fmaxf(sqrtf(ss), eps));
+  const float iq = 1.0f / ((float)hr * fmaxf(sqrtf(ss), eps));
+  if (lane == 0) invq[w] = iq;
+  if (qhat)
+    *reinterpret_cast<uint2*>(qhat + (size_t)w * kHeadDim + 4 * lane) =
+        make_uint2(pack_bf2(a * iq, b * iq), pack_bf2(c * iq, d * iq));
 }
 
 struct SimtArgs {
@@ -156,7 +163,7 @@ msa_status launch_qprep(const RoutePlan& p, float eps, cudaStream_t st) {
   const int64_t zblocks = (zvecs + 255) / 256;
   if (blocks < zblocks) blocks = zblocks < 148 * 4 ? zblocks : 148 * 4;
   cudaError_t e = launch_pdl(qprep_kernel, dim3((unsigned)blocks), dim3(256), 0, st, p.qr, p.n_rows, p.hr, eps,
-                             p.invq, reinterpret_cast<uint4*>(p.zero), zvecs);
+                             p.invq, p.qhat, reinterpret_cast<uint4*>(p.zero), zvecs);
   if (e != cudaSuccess) return cuda_fail(e, "route: query norms");
   return launch_check("route: query norms");
 }

@@ -33,18 +33,18 @@
 #include <cudaTypedefs.h>
 
 #include "msa_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace msa {
 
-__device__ int g_tc_error;  // set by a kernel whose wait ran out; read by msa_sync_check
-
 namespace {
+
+using namespace tc;
 
 constexpr int kHeads = 8;
 constexpr int kTileM = 128;
 constexpr int kThreads = 192;
 constexpr int kEpiWarp0 = 2;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 struct TcArgs {
   const float* invk;        // [C, 8]
@@ -55,90 +55,6 @@ struct TcArgs {
   int n_rows, n_seq, n_tiles, n_nb;
   int32_t q_seq_off[kMaxSeq + 1];
 };
-
-// ------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait; false if it ran out or another role of the CTA gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        atomicExch(&g_tc_error, 1);
-        return false;
-      }
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B,
-// 8-row groups 1024 B apart (stride byte offset), version 1.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
-}
 
 __device__ __forceinline__ int seq_of_row(const int32_t* off, int n_seq, int t) {
   int lo = 0, hi = n_seq - 1;
@@ -158,7 +74,8 @@ struct Cfg {
   static constexpr int kStage = kA + kB;
   static constexpr int kStages = NB <= 16 ? 6 : 5;
   static constexpr int kTmemCols = 2 * kHeads * NB;  // double-buffered 8 heads
-  static constexpr int kSmem = 1024 + kStages * kStage + 4096;  // align slack + stages + barriers, flags, invq
+  static constexpr int kWarpTab = NB * kHeads * 4 + 2 * NB * 4;  // one epilogue warp's column table
+  static constexpr int kSmem = 1024 + kStages * kStage + 256 + 4 * kWarpTab;  // slack, stages, barriers, tables
   // instruction descriptor: D fp32, A/B bf16, both K-major, N = NB, M = 128
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NB >> 3) << 17) |
                                      ((uint32_t)(kTileM >> 4) << 24);
@@ -180,13 +97,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // per row block: query scales [NB][8], and for each column its sequence
-  // (-1 past the last row) and whether a sequence's run ends there
-  float* s_invq = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Each epilogue warp's own table of the current row block: query scales
+  // [NB][8], and per column its sequence (-1 past the last row) and whether a
+  // sequence's run ends there. Private to the warp, so filling it needs only
+  // __syncwarp (no barrier that a warp which gave up could leave waiting).
+  float* s_invq = reinterpret_cast<float*>(smem + C::kStages * C::kStage + 256 +
+                                           (warp >= kEpiWarp0 ? warp - kEpiWarp0 : 0) * C::kWarpTab);
   int* s_seq = reinterpret_cast<int*>(s_invq + NB * kHeads);
   int* s_end = s_seq + NB;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -288,14 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row = 32 * q + lane;           // chunk within the tile
-    const int et = threadIdx.x - 32 * kEpiWarp0;  // 0..127
     auto load_block = [&](int t0) {
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int i = et; i < NB * kHeads; i += 128) {
+      __syncwarp();
+      for (int i = lane; i < NB * kHeads; i += 32) {
         const int t = t0 + i / kHeads;
         s_invq[i] = t < a.n_rows ? a.invq[(size_t)t * kHeads + (i % kHeads)] : 0.f;
       }
-      for (int i = et; i < NB; i += 128) {
+      for (int i = lane; i < NB; i += 32) {
         const int t = t0 + i;
         int sq = -1, end = 0;
         if (t < a.n_rows) {
@@ -305,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_seq[i] = sq;
         s_end[i] = end;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      __syncwarp();
     };
     if (a.n_nb == 1) load_block(0);
     int blk = 0;
