@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 
 def parse_args():
@@ -78,6 +79,18 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor throughput for a kernel timed inside a long step (the
+    sustained figure)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured sustained"
+    return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback sustained"
 
 
 def traffic_for(kernel: str, src: str, workload: str, bytes_scale: float = 1.0):
@@ -404,13 +417,20 @@ class Routed:
     def units_per_step(self) -> float:
         return float(self.w.memory_tokens) * self.S * self.L
 
-    def score_bytes_per_launch(self) -> float:
-        w = self.w
-        C = self.C
+    def scored_chunks(self) -> int:
         if self.run_mode == "sharded":  # the timed launch is shard 0's
             d0, d1 = self.shard_ranges[0]
-            C = int(self.dco[d1] - self.dco[d0])
-        return C * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+            return int(self.dco[d1] - self.dco[d0])
+        return self.C
+
+    def score_bytes_per_launch(self) -> float:
+        w = self.w
+        return self.scored_chunks() * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+
+    def score_flops_per_launch(self) -> float:
+        """The contraction: 2 flops per (query row, chunk, head, dimension)."""
+        w = self.w
+        return 2.0 * self.T * self.scored_chunks() * w.hr * w.d
 
     def check_planted(self):
         """Every layer's routed set must be its planted set (a property of the inputs)."""
@@ -679,20 +699,34 @@ def run_ours(args):
         e2e = run_e2e(eng, w, args, world, unit)
 
     peak, peak_kind = measured_peaks()
-    if w.name == "encode":
-        kbytes = eng.kernel_bytes_per_launch()
-        kname, ksrc = "encode_pool_kernel", "routed_sparse_attention_msa_b200/csrc/encode.cu"
+    # the library picks the many-row (tensor-bound) scorer above 64 query rows
+    many_rows = w.name != "encode" and w.hr == 8 and (
+        args.score_kernel == "tc_rows" or (args.score_kernel == "auto" and eng.T > 64))
+    if many_rows:
+        kflops = eng.score_flops_per_launch()
+        tpeak, tpeak_kind = measured_tensor_peak()
+        achieved = kflops / (kern_avg_ms / 1e3) / 1e12
+        roof = {"kernel": "score_pf_kernel", "bound": "tensor", "achieved": achieved, "peak": tpeak,
+                "unit": "TFLOP/s", "frac": achieved / tpeak, "peak_kind": tpeak_kind,
+                "traffic": traffic_for("score_pf_kernel", "routed_sparse_attention_msa_b200/csrc/score_pf.cu",
+                                       w.name),
+                "algorithmic_flops_per_launch": kflops, "avg_launch_us": kern_avg_ms * 1e3,
+                "launches_per_step": L}
     else:
-        kbytes = eng.score_bytes_per_launch()
-        kname = "score_tc_kernel" if args.score_kernel in ("auto", "tc") else "score_simt_kernel"
-        ksrc = ("routed_sparse_attention_msa_b200/csrc/score_tc.cu" if kname == "score_tc_kernel"
-                else "routed_sparse_attention_msa_b200/csrc/score.cu")
-    achieved = kbytes / (kern_avg_ms / 1e3) / 1e9
-    traffic = traffic_for(kname, ksrc, w.name)
-    roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
-            "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": kern_avg_ms * 1e3,
-            "launches_per_step": L}
+        if w.name == "encode":
+            kbytes = eng.kernel_bytes_per_launch()
+            kname, ksrc = "encode_pool_kernel", "routed_sparse_attention_msa_b200/csrc/encode.cu"
+        else:
+            kbytes = eng.score_bytes_per_launch()
+            kname = "score_tc_kernel" if args.score_kernel in ("auto", "tc") else "score_simt_kernel"
+            ksrc = ("routed_sparse_attention_msa_b200/csrc/score_tc.cu" if kname == "score_tc_kernel"
+                    else "routed_sparse_attention_msa_b200/csrc/score.cu")
+        achieved = kbytes / (kern_avg_ms / 1e3) / 1e9
+        traffic = traffic_for(kname, ksrc, w.name)
+        roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": kern_avg_ms * 1e3,
+                "launches_per_step": L}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:

@@ -80,6 +80,7 @@ _sig("msa_status_string", [ctypes.c_int], ctypes.c_char_p)
 _sig("msa_last_error", [], ctypes.c_char_p)
 _sig("msa_version", [])
 _sig("msa_debug_set_score_kernel", [ctypes.c_int])
+_sig("msa_debug_set_pf_block", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
 _sig("msa_debug_score_events", [P, P], None)
@@ -146,6 +147,12 @@ def score_events(begin, end) -> None:
     """Record torch.cuda.Events ``begin``/``end`` around the scoring kernel of
     the calling thread's next route call (both must already exist)."""
     _lib.msa_debug_score_events(int(begin.cuda_event), int(end.cuda_event))
+
+
+def set_pf_block(rows: int) -> int:
+    """Force the many-row scorer's query-row block (64, 128, 160 or 192; 0 =
+    choose by padding); returns the previous setting. Testing control."""
+    return _lib.msa_debug_set_pf_block(int(rows))
 
 
 def set_score_kernel(which: str) -> str:

@@ -71,18 +71,21 @@ msa_status check_bank(const msa_bank_layer* b, bool need_content) {
 }
 
 struct RouteLayout {
-  size_t invq, qhat, doc_key, topk, total;
+  size_t invq, invq_t, col_code, doc_key, topk, total;
+  int n_rows_pad;
 };
 
-// Workspace of one route call: query scales, the scaled query rows of the
-// many-row scorer (eight routing heads only), document keys, top-k state.
+// Workspace of one route call: query scales (row-major and head-major), the
+// per-row sequence codes, then (cleared before scoring) document keys and
+// top-k state.
 RouteLayout route_layout(const msa_bank_layer* b, int n_seq, int n_rows, int top_k) {
   RouteLayout L;
   int k = top_k < b->n_docs ? top_k : (int)b->n_docs;
+  L.n_rows_pad = (n_rows + 3) & ~3;
   L.invq = 0;
-  L.qhat = align_up((size_t)n_rows * b->hr * sizeof(float), 256);
-  const size_t qhat_bytes = b->hr == 8 ? (size_t)n_rows * b->hr * b->d * sizeof(uint16_t) : 0;
-  L.doc_key = L.qhat + align_up(qhat_bytes, 256);
+  L.invq_t = align_up((size_t)n_rows * b->hr * sizeof(float), 256);
+  L.col_code = L.invq_t + align_up((size_t)L.n_rows_pad * b->hr * sizeof(float), 256);
+  L.doc_key = L.col_code + align_up((size_t)n_rows * sizeof(int32_t), 256);
   L.topk = L.doc_key + align_up((size_t)n_seq * b->n_docs * sizeof(uint32_t), 256);
   L.total = L.topk + topk_workspace(n_seq, b->n_docs, k);
   return L;
@@ -230,7 +233,9 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   p.n_chunks = b->n_chunks; p.n_docs = b->n_docs; p.hr = b->hr; p.n_rows = n_rows; p.n_seq = n_seq;
   for (int i = 0; i <= n_seq; ++i) p.q_seq_off[i] = q_seq_off[i];
   p.invq = reinterpret_cast<float*>(w + L.invq);
-  p.qhat = L.doc_key > L.qhat ? reinterpret_cast<uint16_t*>(w + L.qhat) : nullptr;
+  p.invq_t = reinterpret_cast<float*>(w + L.invq_t);
+  p.col_code = reinterpret_cast<int32_t*>(w + L.col_code);
+  p.n_rows_pad = L.n_rows_pad;
   p.doc_key = reinterpret_cast<uint32_t*>(w + L.doc_key);
   p.zero = w + L.doc_key;
   p.zero_bytes = L.total - L.doc_key;  // a multiple of 256

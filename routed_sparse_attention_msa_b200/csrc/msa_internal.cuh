@@ -99,7 +99,9 @@ struct RoutePlan {
   int32_t hr, n_rows, n_seq;
   int32_t q_seq_off[kMaxSeq + 1];
   float* invq;                 // ws [T, hr]: 1 / (hr * max(||q||, eps))
-  uint16_t* qhat;              // ws [T, hr, d]: bf16(qr * invq) (hr = 8 only, else NULL)
+  float* invq_t;               // ws [hr, Tp]: the same, head-major (Tp = T rounded up to 4)
+  int32_t* col_code;           // ws [T]: row's sequence | 256 if the row ends its sequence
+  int32_t n_rows_pad;          // Tp
   uint32_t* doc_key;           // ws [S, D]: ordered doc scores (0 = none)
   void* zero;                  // ws bytes to clear before scoring (doc keys, top-k state)
   size_t zero_bytes;           // multiple of 16

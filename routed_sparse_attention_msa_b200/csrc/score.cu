@@ -20,30 +20,49 @@
 namespace msa {
 namespace {
 
-// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)) and, when qhat
-// is given, the scaled row bf16(qr * invq) that the many-row scorer
-// contracts; the whole grid also clears the scoring workspace (document keys
-// and top-k state).
-__global__ void qprep_kernel(const uint16_t* __restrict__ qr, int n_rows, int hr, float eps,
-                             float* __restrict__ invq, uint16_t* __restrict__ qhat, uint4* __restrict__ zero,
-                             int64_t zero_vecs) {
+struct QprepArgs {
+  const uint16_t* qr;
+  int n_rows, hr, n_rows_pad, n_seq;
+  float eps;
+  float* invq;       // [T, hr]
+  float* invq_t;     // [hr, Tp]
+  int32_t* col_code; // [T]
+  uint4* zero;
+  int64_t zero_vecs;
+  int32_t q_seq_off[kMaxSeq + 1];
+};
+
+// One warp per (row, head): invq = 1 / (hr * max(||q||, eps)), stored row-major
+// and head-major; per row, its sequence and whether it is the sequence's last
+// row (the column metadata of the many-row scorer). The whole grid also clears
+// the scoring workspace (document keys and top-k state).
+__global__ void qprep_kernel(const __grid_constant__ QprepArgs a) {
   pdl_wait();
   pdl_trigger();
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  for (int64_t i = tid; i < zero_vecs; i += (int64_t)gridDim.x * blockDim.x) zero[i] = make_uint4(0, 0, 0, 0);
+  for (int64_t i = tid; i < a.zero_vecs; i += (int64_t)gridDim.x * blockDim.x) a.zero[i] = make_uint4(0, 0, 0, 0);
   const int lane = threadIdx.x & 31;
   const int w = (int)(tid >> 5);
-  if (w >= n_rows * hr) return;
-  uint2 v = __ldg(reinterpret_cast<const uint2*>(qr + (size_t)w * kHeadDim + 4 * lane));
-  float a = bf_lo(v.x), b = bf_hi(v.x), c = bf_lo(v.y), d = bf_hi(v.y);
-  float ss = a * a + b * b + c * c + d * d;
+  if (w >= a.n_rows * a.hr) return;
+  uint2 v = __ldg(reinterpret_cast<const uint2*>(a.qr + (size_t)w * kHeadDim + 4 * lane));
+  float x0 = bf_lo(v.x), x1 = bf_hi(v.x), x2 = bf_lo(v.y), x3 = bf_hi(v.y);
+  float ss = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float iq = 1.0f / ((float)hr * fmaxf(sqrtf(ss), eps));
-  if (lane == 0) invq[w] = iq;
-  if (qhat)
-    *reinterpret_cast<uint2*>(qhat + (size_t)w * kHeadDim + 4 * lane) =
-        make_uint2(pack_bf2(a * iq, b * iq), pack_bf2(c * iq, d * iq));
+  if (lane == 0) {
+    const float iq = 1.0f / ((float)a.hr * fmaxf(sqrtf(ss), a.eps));
+    const int t = w / a.hr, h = w % a.hr;
+    a.invq[w] = iq;
+    a.invq_t[(size_t)h * a.n_rows_pad + t] = iq;
+    if (h == 0) {
+      int lo = 0, hi = a.n_seq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.q_seq_off[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      a.col_code[t] = lo | (t + 1 == a.q_seq_off[lo + 1] ? 256 : 0);
+    }
+  }
 }
 
 struct SimtArgs {
@@ -162,8 +181,20 @@ msa_status launch_qprep(const RoutePlan& p, float eps, cudaStream_t st) {
   const int64_t zvecs = (int64_t)(p.zero_bytes / 16);
   const int64_t zblocks = (zvecs + 255) / 256;
   if (blocks < zblocks) blocks = zblocks < 148 * 4 ? zblocks : 148 * 4;
-  cudaError_t e = launch_pdl(qprep_kernel, dim3((unsigned)blocks), dim3(256), 0, st, p.qr, p.n_rows, p.hr, eps,
-                             p.invq, p.qhat, reinterpret_cast<uint4*>(p.zero), zvecs);
+  QprepArgs a{};
+  a.qr = p.qr;
+  a.n_rows = p.n_rows;
+  a.hr = p.hr;
+  a.n_rows_pad = p.n_rows_pad;
+  a.n_seq = p.n_seq;
+  a.eps = eps;
+  a.invq = p.invq;
+  a.invq_t = p.invq_t;
+  a.col_code = p.col_code;
+  a.zero = reinterpret_cast<uint4*>(p.zero);
+  a.zero_vecs = zvecs;
+  for (int i = 0; i <= p.n_seq; ++i) a.q_seq_off[i] = p.q_seq_off[i];
+  cudaError_t e = launch_pdl(qprep_kernel, dim3((unsigned)blocks), dim3(256), 0, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "route: query norms");
   return launch_check("route: query norms");
 }

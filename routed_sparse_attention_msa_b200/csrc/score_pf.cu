@@ -4,28 +4,34 @@
 // similarity mean-pooled over heads, then token-wise max; "MSA-arXiv26",
 // 核心方法 — the query scored against every document's pooled routing keys]
 //
-// With hundreds of query rows per call the scoring is a dense contraction
-// (2 x rows x 1,024 flops per pooled chunk), bound by the tensor cores rather
-// than by HBM. Per-head accumulators would cap a pass at 32 query columns
-// (8 heads x 32 x 2 buffers = 512 TMEM columns), so instead both cosine
-// scales are folded into the operands and the head sum becomes part of the
-// contraction:
-//   score(t, c) = sum over (h, i) of Ahat[c, h, i] * Qhat[t, h, i],
-//   Ahat = bf16(kbar_r * invk[c, h]),  Qhat = bf16(qr * invq[t, h])
-// (invq includes the head mean's 1/hr). Rounding the scaled operands to
-// bfloat16 moves a score by about 1e-4, well inside the 1e-3 bar. Qhat is
-// written by the query-norm kernel; Ahat is made in shared memory: a
-// transform warp group rescales each TMA-loaded 128-chunk x 64-dimension
-// stage in place (the 128-byte swizzle permutes 16-byte pieces only within a
-// chunk's own 128-byte row, so a row's scale applies to all of it).
+//   score(s, j) = max over rows t of s and chunks c of j of
+//                 sum_h invk[c,h] * invq[t,h] * (kbar_r[c,h] . qr[t,h])
 //
-// Tile: 128 chunks x NB query rows (NB = 128 or 256) x K = 1,024 in 16
-// stages of 64; one fp32 accumulator of NB TMEM columns, double-buffered.
-// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2-5 transform, 6-9
-// epilogue (a running max per sequence and a per-document flush, as in the
-// decode scorer). Every wait is bounded in time.
+// With hundreds of query rows per call this is a dense contraction (2 x rows
+// x 1,024 flops per pooled chunk) bound by the tensor cores, not by HBM. The
+// decode scorer keeps all eight heads' accumulators in TMEM at once, which
+// caps a pass at 32 query columns; here the heads take turns instead: one
+// K = 128 contraction per head into a 128-chunk x NB-row fp32 accumulator
+// (NB = 64, 128, 160 or 192; two to four of them in TMEM, so the tensor
+// cores run ahead of the epilogue), and the epilogue folds each
+// head into a running sum held in registers,
+//   acc_sum[c, t] += invk[c, h] * invq[t, h] * acc_h[c, t],
+// so the arithmetic is the decode scorer's: bf16 products, fp32 sums, exact
+// cosine scales. After the eighth head the sums are max-reduced over each
+// sequence's columns and over the document's chunks, and flushed with one
+// atomicMax per (sequence, document segment).
+//
+// Warps: 0 TMA producer (one 128 x 64 stage of pooled keys and one NB x 64
+// stage of query rows per mbarrier slot), 1 MMA issuer and TMEM owner, then
+// the epilogue: WQ = 2 or 3 warps per TMEM lane quadrant, each owning NB/WQ
+// columns. A 128 x NB x 16 MMA reads (128 + NB) x 32 bytes of shared memory,
+// so wider blocks need fewer bytes per flop; that, not the TMEM depth, sets
+// the speed of the narrower variants.
+// Per row block an epilogue warp needs its columns' query scales and
+// sequence codes; the query-norm kernel lays both out so that they arrive by
+// a few 16-byte cp.async copies, double-buffered and issued one block ahead.
+// Every wait is bounded in time.
 #include <cuda.h>
-#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include "msa_internal.cuh"
@@ -36,44 +42,48 @@ namespace {
 
 using namespace tc;
 
-constexpr int kM = 128;                      // chunks per tile
-constexpr int kKB = 64;                      // contraction elements per stage (one 128-byte row)
+constexpr int kM = 128;    // chunks per tile
+constexpr int kKB = 64;    // contraction elements per stage (one 128-byte row)
 constexpr int kHeads = 8;
-constexpr int kKSteps = kHeads * 128 / kKB;  // 16
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 6;
+constexpr int kEpiWarp0 = 2;
+constexpr int kSmemMax = 232448;
 
-template <int NB>
+// NB query rows per block, WQ epilogue warps per TMEM lane quadrant.
+template <int NB, int WQ>
 struct PfCfg {
-  static constexpr int kA = kM * kKB * 2;     // 16 KB
-  static constexpr int kB = NB * kKB * 2;     // 16 or 32 KB
+  static constexpr int kEpiWarps = 4 * WQ;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kA = kM * kKB * 2;            // 16 KB
+  static constexpr int kB = NB * kKB * 2;
   static constexpr int kStage = kA + kB;
-  static constexpr int kStages = 196608 / kStage;  // 4 or 6
-  static constexpr int kTmemCols = 2 * NB;
-  static constexpr int kWarpTab = NB * 2;     // int16 per column
-  static constexpr int kSmem = 1024 + kStages * kStage + 256 + 4 * kWarpTab;
+  static constexpr int kTBuf = 512 / NB < 4 ? 512 / NB : 4;  // TMEM accumulators
+  static constexpr int kTmemCols = 512;
+  static constexpr int kCols = NB / WQ;              // columns per epilogue warp
+  static constexpr int kChunks = (kCols + 31) / 32;  // 32-column groups of the flush
+  // one epilogue warp's tables: two buffers of {query scales [h][col],
+  // column codes [col]}, key scales [h][lane], document ids [lane]
+  static constexpr int kIqTab = kHeads * kCols * 4;
+  static constexpr int kColTab = kIqTab + kCols * 4;
+  static constexpr int kWarpTab = 2 * kColTab + kHeads * 32 * 4 + 32 * 4;
+  static constexpr int kFixed = 1024 + 256 + kEpiWarps * kWarpTab;
+  static constexpr int kStages = (kSmemMax - kFixed) / kStage < 8 ? (kSmemMax - kFixed) / kStage : 8;
+  static constexpr int kSmem = kFixed + kStages * kStage;
   // instruction descriptor: D fp32, A/B bf16, both K-major, N = NB, M = 128
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NB >> 3) << 17) |
                                      ((uint32_t)(kM >> 4) << 24);
+  static_assert(kCols % 16 == 0 && kCols * WQ == NB && kStages >= 3 && kTBuf >= 2, "tile configuration");
 };
 
 struct PfArgs {
   const float* invk;         // [C, 8]
   const int32_t* chunk_doc;  // [C]
+  const float* invq_t;       // [8, Tp]
+  const int32_t* col_code;   // [T]
   uint32_t* doc_key;         // [S, D]
   int64_t n_chunks, n_docs;
-  int n_rows, n_seq, n_tiles, n_nb;
-  int32_t q_seq_off[kMaxSeq + 1];
+  int n_rows, n_rows_pad, n_tiles, n_nb;
 };
-
-__device__ __forceinline__ int seq_of_row(const int32_t* off, int n_seq, int t) {
-  int lo = 0, hi = n_seq - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= t) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -82,44 +92,74 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Two bf16 (packed) times a scale, rounded back to a bf16 pair.
-__device__ __forceinline__ uint32_t scale_bf2(uint32_t w, float s) {
-  const __nv_bfloat162 r = __floats2bfloat162_rn(bf_lo(w) * s, bf_hi(w) * s);
-  return *reinterpret_cast<const uint32_t*>(&r);
+// 16-byte global -> shared copy that bypasses registers; the bytes past
+// src_bytes (0..16) are written as zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Two IEEE fp32 operations in one instruction (Blackwell packed fp32):
+// d = a * b + c and d = a * b on a pair of lanes, rounded like fmaf / a * b.
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, C, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\tmov.b64 C, {%6, %7};\n\t"
+      "fma.rn.f32x2 D, A, B, C;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mul.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
-template <int NB>
-__global__ void __launch_bounds__(kThreads, 1)
+// Maximum of W consecutive values (W a power of two, a balanced tree).
+template <int W>
+__device__ __forceinline__ float max_tree(const float* x) {
+  float t[W / 2];
+#pragma unroll
+  for (int j = 0; j < W / 2; ++j) t[j] = fmaxf(x[j], x[j + W / 2]);
+#pragma unroll
+  for (int w = W / 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+  return t[0];
+}
+
+template <int NB, int WQ>
+__global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
     score_pf_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ PfArgs a) {
-  using C = PfCfg<NB>;
+  using C = PfCfg<NB, WQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
-  uint64_t* ready = full + C::kStages;
-  uint64_t* empty = ready + C::kStages;
+  uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
+  uint64_t* tempty = tfull + C::kTBuf;
+  uint64_t* mma_done = tempty + C::kTBuf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* warp_tabs = smem + C::kStages * C::kStage + 256;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // An epilogue warp's own column table for the current row block: the
-  // column's sequence, +256 where a sequence's run ends, -1 past the last row.
-  int16_t* s_col = reinterpret_cast<int16_t*>(smem + C::kStages * C::kStage + 256 +
-                                              (warp >= kEpiWarp0 ? warp - kEpiWarp0 : 0) * C::kWarpTab);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&ready[s]), 128);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kTBuf; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 128);
+      mbar_init(smem_u32(&tempty[b]), C::kEpiThreads);
     }
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
@@ -134,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();
+  pdl_wait();  // the prologue above overlapped the previous kernel's tail
   pdl_trigger();
 
   if (warp == 0) {
@@ -145,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x)
         for (int nb = 0; nb < a.n_nb && ok; ++nb)
-          for (int kb = 0; kb < kKSteps; ++kb) {
+          for (int kb = 0; kb < 2 * kHeads; ++kb) {
             if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) { ok = false; break; }
             const uint32_t st = smem_u32(stages + s * C::kStage);
             const uint32_t fb = smem_u32(&full[s]);
@@ -170,137 +210,192 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
     if (lane == 0) {
-      int s = 0, blk = 0;
-      uint32_t ph = 0;
+      int s = 0, b = 0;
+      uint32_t ph = 0, tph = 0;  // stage ring and TMEM ring phases
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x) {
-        for (int nb = 0; nb < a.n_nb && ok; ++nb, ++blk) {
-          const int b = blk & 1;
-          if (!mbar_wait(smem_u32(&tempty[b]), ((blk >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(b * NB);
-          for (int kb = 0; kb < kKSteps; ++kb) {
-            if (!mbar_wait(smem_u32(&ready[s]), ph, abort_flag)) { ok = false; break; }
+      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x)
+        for (int nb = 0; nb < a.n_nb && ok; ++nb)
+          for (int h = 0; h < kHeads && ok; ++h) {
+            if (!mbar_wait(smem_u32(&tempty[b]), tph ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t st = smem_u32(stages + s * C::kStage);
+            const uint32_t d = tmem + (uint32_t)(b * NB);
+            for (int ks = 0; ks < 2; ++ks) {
+              if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t st = smem_u32(stages + s * C::kStage);
 #pragma unroll
-            for (int k = 0; k < kKB / 16; ++k)
-              tc_mma(d, sw128_desc(st + k * 32), sw128_desc(st + C::kA + k * 32), C::kIdesc, (kb | k) ? 1u : 0u);
-            tc_commit(smem_u32(&empty[s]));
-            if (++s == C::kStages) { s = 0; ph ^= 1; }
+              for (int k = 0; k < kKB / 16; ++k)
+                tc_mma(d, sw128_desc(st + k * 32), sw128_desc(st + C::kA + k * 32), C::kIdesc, (ks | k) ? 1u : 0u);
+              tc_commit(smem_u32(&empty[s]));
+              if (++s == C::kStages) { s = 0; ph ^= 1; }
+            }
+            if (ok) tc_commit(smem_u32(&tfull[b]));
+            if (++b == C::kTBuf) { b = 0; tph ^= 1; }
           }
-          if (ok) tc_commit(smem_u32(&tfull[b]));
-        }
-      }
       // Every MMA this thread issued has completed once mma_done flips.
       tc_commit(smem_u32(mma_done));
       const uint64_t t0 = globaltimer();
       while (!mbar_try(smem_u32(mma_done), 0) && globaltimer() - t0 < kWaitLimitNs) {
       }
     }
-  } else if (warp < kEpiWarp0) {
-    // ---------------------------------------- transform: A *= invk[c, h]
-    const int r = threadIdx.x - 64;  // chunk row within the tile
-    int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x) {
-      const int64_t c = (int64_t)tile * kM + r;
-      float ik[kHeads];
-      if (c < a.n_chunks) {
-        const float4 u0 = __ldg(reinterpret_cast<const float4*>(a.invk + c * kHeads));
-        const float4 u1 = __ldg(reinterpret_cast<const float4*>(a.invk + c * kHeads + 4));
-        ik[0] = u0.x; ik[1] = u0.y; ik[2] = u0.z; ik[3] = u0.w;
-        ik[4] = u1.x; ik[5] = u1.y; ik[6] = u1.z; ik[7] = u1.w;
-      } else {
-#pragma unroll
-        for (int h = 0; h < kHeads; ++h) ik[h] = 0.f;
-      }
-      for (int nb = 0; nb < a.n_nb && ok; ++nb)
-#pragma unroll
-        for (int kb = 0; kb < kKSteps; ++kb) {
-          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) { ok = false; break; }
-          const float sc = ik[kb >> 1];  // two 64-dimension stages per head
-          // The row's eight 16-byte pieces are visited starting at piece
-          // r mod 8, so the eight rows of each 8-thread access phase touch
-          // eight different bank groups (the scale is the same for all).
-          uint4* row = reinterpret_cast<uint4*>(stages + s * C::kStage + r * 128);
-          uint4 w[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) w[u] = row[u ^ (r & 7)];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            row[u ^ (r & 7)] = make_uint4(scale_bf2(w[u].x, sc), scale_bf2(w[u].y, sc), scale_bf2(w[u].z, sc),
-                                          scale_bf2(w[u].w, sc));
-          fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
-          mbar_arrive(smem_u32(&ready[s]));
-          if (++s == C::kStages) { s = 0; ph ^= 1; }
-        }
-    }
   } else {
     // --------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quadrant of this warp
-    const int row = 32 * q + lane;
-    int blk = 0;
+    const int ew = warp - kEpiWarp0;        // 0 .. 4 WQ - 1
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int col0 = (ew >> 2) * C::kCols;  // this warp's columns within the row block
+    const int row = 32 * q + lane;          // chunk within the tile
+    // This warp's tables live in shared memory: the L1 left beside ~200 KB of
+    // stages is small, and the head loop must not wait on L2.
+    uint8_t* wt = warp_tabs + ew * C::kWarpTab;
+    float* s_ik = reinterpret_cast<float*>(wt + 2 * C::kColTab);              // [h][lane]
+    int* s_doc = reinterpret_cast<int*>(wt + 2 * C::kColTab + kHeads * 128);  // [lane]
+    auto iq_tab = [&](int k) { return reinterpret_cast<float*>(wt + k * C::kColTab); };
+    auto code_tab = [&](int k) { return reinterpret_cast<int32_t*>(wt + k * C::kColTab + C::kIqTab); };
+    // Query scales [h][col] and column codes of row block nbx into buffer k,
+    // asynchronously; bytes past the last row arrive as zeros.
+    auto fill = [&](int nbx, int k) {
+      const int tw = nbx * NB + col0;
+      const int left = a.n_rows - tw;  // valid columns from tw on
+      float* dq = iq_tab(k);
+      for (int i = lane; i < kHeads * C::kCols / 4; i += 32) {
+        const int h = i / (C::kCols / 4), j = 4 * (i % (C::kCols / 4));
+        const int nbytes = left - j >= 4 ? 16 : left - j > 0 ? 4 * (left - j) : 0;
+        cp_async16(dq + h * C::kCols + j, nbytes ? a.invq_t + (size_t)h * a.n_rows_pad + tw + j : a.invq_t, nbytes);
+      }
+      int32_t* dc = code_tab(k);
+      for (int j = 4 * lane; j < C::kCols; j += 128) {
+        const int nbytes = left - j >= 4 ? 16 : left - j > 0 ? 4 * (left - j) : 0;
+        cp_async16(dc + j, nbytes ? a.col_code + tw + j : a.col_code, nbytes);
+      }
+      cp_async_commit();
+    };
+    fill(0, 0);
+    int b = 0, blk = 0;
+    uint32_t tph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x) {
       const int64_t c = (int64_t)tile * kM + row;
       const bool valid = c < a.n_chunks;
-      const int doc = valid ? __ldg(a.chunk_doc + c) : -1;
-      // lanes whose right-hand neighbour at distance o is in the same document
-      unsigned same = 0;
-#pragma unroll
-      for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
-        const int dn = __shfl_down_sync(0xffffffffu, doc, o);
-        if (lane + o < 32 && dn == doc) same |= 1u << i;
-      }
-      const int doc_up = __shfl_up_sync(0xffffffffu, doc, 1);
-      const bool head = valid && (lane == 0 || doc_up != doc);
-      for (int nb = 0; nb < a.n_nb; ++nb, ++blk) {
-        const int b = blk & 1;
-        const int t0 = nb * NB;
-        __syncwarp();
-        for (int i = lane; i < NB; i += 32) {
-          const int t = t0 + i;
-          int v = -1;
-          if (t < a.n_rows) {
-            const int sq = seq_of_row(a.q_seq_off, a.n_seq, t);
-            const bool end = (t + 1 == a.q_seq_off[sq + 1]) || (i == NB - 1);
-            v = sq | (end ? 256 : 0);
-          }
-          s_col[i] = (int16_t)v;
+      {  // key scales and document of this lane's chunk (each lane reads only its own slots)
+        float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+        int d = -1;
+        if (valid) {
+          u0 = __ldg(reinterpret_cast<const float4*>(a.invk + c * kHeads));
+          u1 = __ldg(reinterpret_cast<const float4*>(a.invk + c * kHeads + 4));
+          d = __ldg(a.chunk_doc + c);
         }
+        s_ik[0 * 32 + lane] = u0.x; s_ik[1 * 32 + lane] = u0.y; s_ik[2 * 32 + lane] = u0.z;
+        s_ik[3 * 32 + lane] = u0.w; s_ik[4 * 32 + lane] = u1.x; s_ik[5 * 32 + lane] = u1.y;
+        s_ik[6 * 32 + lane] = u1.z; s_ik[7 * 32 + lane] = u1.w;
+        s_doc[lane] = d;
+      }
+
+      for (int nb = 0; nb < a.n_nb && ok; ++nb, ++blk) {
+        const int tw = nb * NB + col0;  // first query row of this warp's columns
+        const int cur = a.n_nb > 1 ? (blk & 1) : 0;
+        const bool prefetch = a.n_nb > 1 && (nb + 1 < a.n_nb || tile + (int)gridDim.x < a.n_tiles);
+        cp_async_wait_all();
         __syncwarp();
-        if (!mbar_wait(smem_u32(&tfull[b]), (blk >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        float m = -INFINITY;
-#pragma unroll 1
-        for (int j0 = 0; j0 < NB; j0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * NB + j0), v);
-          tmem_ld_wait();
-          if (j0 + 32 >= NB) {  // the whole accumulator is in registers
-            tc_fence_before();
-            mbar_arrive(smem_u32(&tempty[b]));
-          }
+        const float* iq = iq_tab(cur);
+        const int32_t* s_code = code_tab(cur);
+
+        float acc[C::kCols];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int cv = s_col[j0 + j];  // uniform across the warp
-            if (cv < 0) break;
-            m = fmaxf(m, v[j]);
-            if (cv & 256) {
+        for (int j = 0; j < C::kCols; ++j) acc[j] = 0.f;
+        for (int h = 0; h < kHeads; ++h) {
+          if (!mbar_wait(smem_u32(&tfull[b]), tph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const float kh = s_ik[h * 32 + lane];
+          const float2 k2 = make_float2(kh, kh);
+          const float* iqh = iq + h * C::kCols;
 #pragma unroll
-              for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
-                const float mo = __shfl_down_sync(0xffffffffu, m, o);
-                if (same & (1u << i)) m = fmaxf(m, mo);
-              }
-              if (head) atomicMax(a.doc_key + (size_t)(cv & 255) * a.n_docs + doc, ord_f32(m));
-              m = -INFINITY;
+          for (int cc = 0; cc < C::kCols / 16; ++cc) {
+            float v[16];
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * NB + col0 + cc * 16), v);
+            tmem_ld_wait();
+            if (cc == C::kCols / 16 - 1) {  // this warp's part of the accumulator is in registers
+              tc_fence_before();
+              mbar_arrive(smem_u32(&tempty[b]));
+            }
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(iqh + cc * 16 + 4 * j4);
+              float* ac = acc + cc * 16 + 4 * j4;
+              const float2 lo = fma_f32x2(make_float2(v[4 * j4], v[4 * j4 + 1]),
+                                          mul_f32x2(k2, make_float2(s4.x, s4.y)), make_float2(ac[0], ac[1]));
+              const float2 hi = fma_f32x2(make_float2(v[4 * j4 + 2], v[4 * j4 + 3]),
+                                          mul_f32x2(k2, make_float2(s4.z, s4.w)), make_float2(ac[2], ac[3]));
+              ac[0] = lo.x; ac[1] = lo.y; ac[2] = hi.x; ac[3] = hi.y;
             }
           }
+          if (++b == C::kTBuf) { b = 0; tph ^= 1; }
+          // the next row block's tables, once this head's TMEM is released
+          if (h == 0 && prefetch) fill(nb + 1 < a.n_nb ? nb + 1 : 0, cur ^ 1);
+        }
+        if (!ok) break;
+
+        // Max over each sequence's columns, then over the document's chunks
+        // (segmented warp max), one atomicMax per segment head. Column
+        // metadata is uniform across the warp; valid columns form a prefix,
+        // and this warp's last valid column also closes a (partial) run.
+        const int nvalid = a.n_rows - tw < C::kCols ? a.n_rows - tw : C::kCols;
+        const int doc = s_doc[lane];
+        // lanes whose right-hand neighbour at distance o is in the same document
+        unsigned same = 0;
+#pragma unroll
+        for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
+          const int dn = __shfl_down_sync(0xffffffffu, doc, o);
+          if (lane + o < 32 && dn == doc) same |= 1u << i;
+        }
+        const int doc_up = __shfl_up_sync(0xffffffffu, doc, 1);
+        const bool head = valid && (lane == 0 || doc_up != doc);
+        float m = -INFINITY;
+        auto flush = [&](float x, int sq) {
+#pragma unroll
+          for (int o = 1, i = 0; o < 32; o <<= 1, ++i) {
+            const float xo = __shfl_down_sync(0xffffffffu, x, o);
+            if (same & (1u << i)) x = fmaxf(x, xo);
+          }
+          if (head) atomicMax(a.doc_key + (size_t)sq * a.n_docs + doc, ord_f32(x));
+        };
+#pragma unroll
+        for (int cc = 0; cc < C::kChunks; ++cc) {
+          const int width = cc == C::kChunks - 1 ? C::kCols - 32 * cc : 32;  // columns in this group
+          const int nv = nvalid - cc * 32;  // valid columns in this group (if < width)
+          if (nv <= 0) break;
+          const unsigned vm = nv >= 32 ? 0xffffffffu : (1u << nv) - 1u;
+          const int code = lane < width ? s_code[cc * 32 + lane] : 0;
+          unsigned em = __ballot_sync(0xffffffffu, lane < nv && (code & 256));
+          if (nv <= width) em |= 1u << (nv - 1);
+          if (width == 32 && vm == 0xffffffffu && (em & 0x7fffffffu) == 0) {  // one run through the group
+            const float x = fmaxf(m, max_tree<32>(acc + (cc * 32 < C::kCols - 31 ? cc * 32 : 0)));
+            if (em) {
+              flush(x, __shfl_sync(0xffffffffu, code, 31) & 255);
+              m = -INFINITY;
+            } else {
+              m = x;
+            }
+            continue;
+          }
+          int lo = 0;
+          while (em) {
+            const int hi = __ffs(em) - 1;
+            em &= em - 1;
+            float x = m;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (cc * 32 + j < C::kCols && j >= lo && j <= hi) x = fmaxf(x, acc[cc * 32 + j]);
+            flush(x, __shfl_sync(0xffffffffu, code, hi) & 255);
+            m = -INFINITY;
+            lo = hi + 1;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (cc * 32 + j < C::kCols && j >= lo && ((vm >> j) & 1u)) m = fmaxf(m, acc[cc * 32 + j]);
         }
       }
     }
+    cp_async_wait_all();  // no table copy may still be in flight at exit
   }
 
   tc_fence_before();
@@ -336,33 +431,35 @@ bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NB>
+template <int NB, int WQ>
 msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
-  using C = PfCfg<NB>;
+  using C = PfCfg<NB, WQ>;
   CUtensorMap ma, mb;
-  if (!make_map_2d(&ma, p.kbar_r, p.n_chunks, kM) || !make_map_2d(&mb, p.qhat, p.n_rows, NB))
+  if (!make_map_2d(&ma, p.kbar_r, p.n_chunks, kM) || !make_map_2d(&mb, p.qr, p.n_rows, NB))
     return fail(MSA_ERR_CUDA, "route: cannot encode TMA tensor maps (cuTensorMapEncodeTiled)");
   PfArgs a{};
   a.invk = p.kr_inv_norm;
   a.chunk_doc = p.chunk_doc;
+  a.invq_t = p.invq_t;
+  a.col_code = p.col_code;
   a.doc_key = p.doc_key;
   a.n_chunks = p.n_chunks;
   a.n_docs = p.n_docs;
   a.n_rows = p.n_rows;
-  a.n_seq = p.n_seq;
+  a.n_rows_pad = p.n_rows_pad;
   a.n_tiles = (int)((p.n_chunks + kM - 1) / kM);
   a.n_nb = (p.n_rows + NB - 1) / NB;
-  for (int i = 0; i <= p.n_seq; ++i) a.q_seq_off[i] = p.q_seq_off[i];
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(score_pf_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e =
+        cudaFuncSetAttribute(score_pf_kernel<NB, WQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return cuda_fail(e, "route: many-row scorer shared memory");
     attr_set = true;
   }
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = a.n_tiles < sms ? a.n_tiles : sms;
-  cudaError_t e = launch_pdl(score_pf_kernel<NB>, dim3(grid), dim3(kThreads), (size_t)C::kSmem, st, ma, mb, a);
+  cudaError_t e = launch_pdl(score_pf_kernel<NB, WQ>, dim3(grid), dim3(C::kThreads), (size_t)C::kSmem, st, ma, mb, a);
   if (e != cudaSuccess) return cuda_fail(e, "route: score (tensor cores, many rows)");
   return launch_check("route: score (tensor cores, many rows)");
 }
@@ -370,15 +467,45 @@ msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
 }  // namespace
 
 bool score_pf_supported(const RoutePlan& p) {
-  // eight routing heads (K = 1,024); 16-byte aligned tensor-map bases
-  return p.hr == kHeads && p.n_chunks > 0 && p.qhat != nullptr &&
-         (reinterpret_cast<uintptr_t>(p.kbar_r) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.qhat) & 15) == 0;
+  // eight routing heads; 16-byte aligned tensor-map bases
+  return p.hr == kHeads && p.n_chunks > 0 && (reinterpret_cast<uintptr_t>(p.kbar_r) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(p.qr) & 15) == 0;
 }
 
+int g_pf_block = 0;  // testing control: force a row block (0 = choose)
+
 msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st) {
-  if (p.n_rows <= 128) return launch_nb<128>(p, st);
-  return launch_nb<256>(p, st);
+  // The row block with the least estimated time: padded columns times the
+  // time per column of each variant (measured on B200 with a 161K-chunk bank;
+  // wider blocks read fewer shared-memory bytes per flop).
+  const int cand[4] = {64, 128, 160, 192};
+  const int per_col[4] = {81, 45, 40, 36};
+  int best = 128;
+  int64_t best_cost = INT64_MAX;
+  for (int i = 0; i < 4; ++i) {
+    const int64_t blocks = (p.n_rows + cand[i] - 1) / cand[i];
+    const int64_t cost = blocks * cand[i] * per_col[i];
+    if (cost < best_cost) { best_cost = cost; best = cand[i]; }
+  }
+  if (g_pf_block) best = g_pf_block;
+  if (best == 64) return launch_nb<64, 2>(p, st);
+  if (best == 160) return launch_nb<160, 2>(p, st);
+  if (best == 192) return launch_nb<192, 3>(p, st);
+  return launch_nb<128, 2>(p, st);
 }
+
+}  // namespace msa
+
+// Forces the many-row scorer's row block (64, 128, 160 or 192; 0 = choose by
+// padding) for later route calls in this process; returns the previous
+// setting. A testing and benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_pf_block(int nb) {
+  const int old = msa::g_pf_block;
+  if (nb == 0 || nb == 64 || nb == 128 || nb == 160 || nb == 192) msa::g_pf_block = nb;
+  return old;
+}
+
+namespace msa {
 
 int pf_error_take() {
   int v = 0;
