@@ -44,6 +44,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
     p.add_argument("--score-kernel", choices=["auto", "simt", "tc", "tc_rows"], default="auto")
+    p.add_argument("--attend-kernel", choices=["auto", "split", "tc"], default="auto")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
     p.add_argument("--content-layers", type=int, default=1,
@@ -548,7 +549,7 @@ def config_of(w, eng, args, extra=None):
                     "top_k": w.top_k, "hq": w.hq, "hkv": w.hkv, "local_tokens": w.loc_len,
                     "content": "pinned_host" if w.content_on_host else "hbm",
                     "gather": args.gather if w.content_on_host else "hbm_index",
-                    "score_kernel": args.score_kernel})
+                    "score_kernel": args.score_kernel, "attend_kernel": args.attend_kernel})
     else:
         cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
     cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
@@ -609,6 +610,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
     import routed_sparse_attention_msa_b200 as msa
     msa.set_score_kernel(args.score_kernel)
+    msa.set_attend_kernel(args.attend_kernel)
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs

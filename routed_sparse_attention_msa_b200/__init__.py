@@ -81,6 +81,7 @@ _sig("msa_last_error", [], ctypes.c_char_p)
 _sig("msa_version", [])
 _sig("msa_debug_set_score_kernel", [ctypes.c_int])
 _sig("msa_debug_set_pf_block", [ctypes.c_int])
+_sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
 _sig("msa_debug_score_events", [P, P], None)
@@ -147,6 +148,13 @@ def score_events(begin, end) -> None:
     """Record torch.cuda.Events ``begin``/``end`` around the scoring kernel of
     the calling thread's next route call (both must already exist)."""
     _lib.msa_debug_score_events(int(begin.cuda_event), int(end.cuda_event))
+
+
+def set_attend_kernel(which: str) -> str:
+    """'auto', 'split' (split-K decoding kernel) or 'tc' (tensor cores, many
+    rows); returns the previous setting. Testing control."""
+    names = ["auto", "split", "tc"]
+    return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
 
 
 def set_pf_block(rows: int) -> int:

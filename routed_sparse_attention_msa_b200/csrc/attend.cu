@@ -28,7 +28,7 @@
 
 #include <algorithm>
 
-#include "msa_internal.cuh"
+#include "attend_params.cuh"
 
 namespace msa {
 namespace {
@@ -37,31 +37,6 @@ constexpr int kMaxVec = 16;    // query vectors per CTA (group x rows): 4, 8 or 
 constexpr int kKeyBlock = 64;  // keys per block
 constexpr int kThreads = 128;
 constexpr int kPad = 132;      // fp32 row stride in shared memory (bank-conflict free)
-
-struct AttnParams {
-  const uint16_t* q;
-  const uint16_t* k_loc;
-  const uint16_t* v_loc;
-  const uint16_t* mem_k;
-  const uint16_t* mem_v;
-  const int64_t* sel_off;
-  const int64_t* sel_chunk;
-  float* qrot;      // [n_q, hq, d]
-  float* krot;      // [n_loc, hkv, d]
-  float* part_o;    // [n_q, hq, splits, d]
-  float2* part_ml;  // [n_q, hq, splits]
-  unsigned* tickets;  // [n_tiles * hkv]
-  uint16_t* out;
-  float* out_f32;
-  float* lse;
-  int n_seq, n_q, n_loc, hq, hkv, group, rt, n_splits, n_tiles;
-  float scale;
-  double pos_offset, log2_theta;
-  int32_t q_seq_off[kMaxSeq + 1];
-  int32_t q_start[kMaxSeq];
-  int32_t loc_off[kMaxSeq + 1];
-  int32_t tile_off[kMaxSeq + 1];
-};
 
 template <int VEC>
 struct Smem {
@@ -74,30 +49,29 @@ struct Smem {
   bool last;
 };
 
-__device__ __forceinline__ int seq_of(const int32_t* off, int n_seq, int x) {
-  int lo = 0, hi = n_seq - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= x) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
+// One thread per (row, group of 4 heads, pair) of the query rows, then of the
+// local keys: the angle depends on the position and the pair only, so it is
+// formed once per thread and applied to the group's heads (loads issued
+// together).
+constexpr int kRopeHeads = 4;
 
-// One thread per (row, head, pair) of the query rows, then of the local keys.
 __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
   pdl_wait();
   pdl_trigger();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < (int64_t)p.n_tiles * p.hkv) p.tickets[idx] = 0u;
-  const int64_t nq = (int64_t)p.n_q * p.hq * 64;
-  const int64_t nk = (int64_t)p.n_loc * p.hkv * 64;
+  const int gq = (p.hq + kRopeHeads - 1) / kRopeHeads, gk = (p.hkv + kRopeHeads - 1) / kRopeHeads;
+  const int64_t nq = (int64_t)p.n_q * gq * 64;
+  const int64_t nk = (int64_t)p.n_loc * gk * 64;
   if (idx >= nq + nk) return;
   const bool is_q = idx < nq;
   const int64_t j = is_q ? idx : idx - nq;
   const int heads = is_q ? p.hq : p.hkv;
+  const int groups = is_q ? gq : gk;
   const int i = (int)(j & 63);
-  const int64_t rh = j >> 6;
-  const int row = (int)(rh / heads);
+  const int64_t rg = j >> 6;
+  const int row = (int)(rg / groups);
+  const int h0 = (int)(rg % groups) * kRopeHeads;
   double pos;
   if (is_q) {
     const int s = seq_of(p.q_seq_off, p.n_seq, row);
@@ -106,17 +80,29 @@ __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
     const int s = seq_of(p.loc_off, p.n_seq, row);
     pos = p.pos_offset + (double)(row - p.loc_off[s]);
   }
-  const uint16_t* src = (is_q ? p.q : p.k_loc) + rh * kHeadDim;
-  float* dst = (is_q ? p.qrot : p.krot) + rh * kHeadDim;
   const double w = exp2(-2.0 * (double)i / (double)kHeadDim * p.log2_theta);
   const double ang = pos * w;
   const double two_pi = 6.283185307179586476925286766559;
   const float r = (float)(ang - two_pi * rint(ang / two_pi));  // in [-pi, pi]
   float sn, cs;
   sincosf(r, &sn, &cs);
-  const float x0 = bf1(src[i]), x1 = bf1(src[i + 64]);
-  dst[i] = x0 * cs - x1 * sn;
-  dst[i + 64] = x0 * sn + x1 * cs;
+  const size_t base = ((size_t)row * heads + h0) * kHeadDim + i;
+  const uint16_t* src = (is_q ? p.q : p.k_loc) + base;
+  float* dst = (is_q ? p.qrot : p.krot) + base;
+  float x0[kRopeHeads], x1[kRopeHeads];
+#pragma unroll
+  for (int u = 0; u < kRopeHeads; ++u) {
+    const bool in = h0 + u < heads;
+    x0[u] = in ? bf1(src[u * kHeadDim]) : 0.f;
+    x1[u] = in ? bf1(src[u * kHeadDim + 64]) : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < kRopeHeads; ++u) {
+    if (h0 + u < heads) {
+      dst[u * kHeadDim] = x0[u] * cs - x1[u] * sn;
+      dst[u * kHeadDim + 64] = x0[u] * sn + x1[u] * cs;
+    }
+  }
 }
 
 // VEC query vectors per CTA: logits give each key two threads of VEC/2
@@ -720,15 +706,40 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_dkdv_kernel(const __grid_
 
 struct Shape {
   int vec, rt, n_tiles, n_splits, n_loc;
+  bool tc;  // tensor-core kernel (many rows per sequence)
 };
 
-Shape plan(const msa_attend_args& a) {
+int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores (testing control)
+
+// allow_tc: the forward may take the tensor-core kernel when the query
+// vectors of a sequence fill at least half of its 128-vector tile.
+Shape plan(const msa_attend_args& a, bool allow_tc) {
   Shape sh;
   const int group = a.hq / a.hkv;
   int max_rows = 1;
   for (int s = 0; s < a.n_seq; ++s) {
     const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
     max_rows = rows > max_rows ? rows : max_rows;
+  }
+  sh.tc = allow_tc && g_attend_kernel != 1 && kAttnTcVec % group == 0 &&
+          (g_attend_kernel == 2 || max_rows * group >= kAttnTcVec / 2);
+  if (sh.tc) {
+    sh.vec = kAttnTcVec;
+    sh.rt = kAttnTcVec / group;
+    sh.n_tiles = 0;
+    int max_loc = 0;
+    for (int s = 0; s < a.n_seq; ++s) {
+      sh.n_tiles += (a.q_seq_off[s + 1] - a.q_seq_off[s] + sh.rt - 1) / sh.rt;
+      max_loc = std::max(max_loc, a.loc_off[s + 1] - a.loc_off[s]);
+    }
+    sh.n_loc = a.loc_off[a.n_seq];
+    // split the 64-key blocks across CTAs while (tiles x kv heads) is under one wave
+    const int64_t ctas = (int64_t)sh.n_tiles * a.hkv;
+    const int64_t blocks = (a.max_sel + max_loc + 63) / 64;
+    int64_t splits = ctas > 0 ? (148 + ctas - 1) / ctas : 1;
+    splits = std::min<int64_t>(std::min<int64_t>(splits, blocks), 64);
+    sh.n_splits = (int)std::max<int64_t>(splits, 1);
+    return sh;
   }
   // query vectors per CTA: the GQA group times enough rows, 4 to 16
   sh.vec = 4;
@@ -788,7 +799,7 @@ msa_status launch_vec(const AttnParams& P, dim3 grid, cudaStream_t st) {
 }  // namespace
 
 size_t attend_workspace(const msa_attend_args& a, int* n_splits_out) {
-  const Shape sh = plan(a);
+  const Shape sh = plan(a, true);
   if (n_splits_out) *n_splits_out = sh.n_splits;
   return layout(a, sh).total;
 }
@@ -823,7 +834,8 @@ void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, cha
 }
 
 msa_status launch_rope(const AttnParams& P, const msa_attend_args& a, const Shape& sh, cudaStream_t st) {
-  int64_t n = (int64_t)a.n_q * a.hq * 64 + (int64_t)sh.n_loc * a.hkv * 64;
+  const int gq = (a.hq + kRopeHeads - 1) / kRopeHeads, gk = (a.hkv + kRopeHeads - 1) / kRopeHeads;
+  int64_t n = (int64_t)a.n_q * gq * 64 + (int64_t)sh.n_loc * gk * 64;
   const int64_t nt = (int64_t)sh.n_tiles * a.hkv;
   if (n < nt) n = nt;
   cudaError_t e = launch_pdl(rope_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, P);
@@ -850,12 +862,13 @@ msa_status launch_bwd_dq(const AttnParams& P, const float* dout, const float* Dv
 }  // namespace
 
 msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
-  const Shape sh = plan(a);
+  const Shape sh = plan(a, true);
   const Layout L = layout(a, sh);
   AttnParams P{};  // kernel parameter block (4.3 KB: large kernel parameters, CUDA >= 12.1)
   fill_params(a, sh, L, reinterpret_cast<char*>(ws), P);
   msa_status s = launch_rope(P, a, sh, st);
   if (s != MSA_OK) return s;
+  if (sh.tc) return launch_attend_tc(P, st);
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
     case 4: return launch_vec<4>(P, grid, st);
@@ -865,14 +878,14 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
 }
 
 size_t attend_backward_workspace(const msa_attend_args& a) {
-  const Shape sh = plan(a);
+  const Shape sh = plan(a, false);
   const Layout L = layout(a, sh);
   return L.total + align_up((size_t)a.n_q * a.hq * sizeof(float), 256);
 }
 
 msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, float* dq, float* dk_loc,
                                   float* dv_loc, float* dmem_k, float* dmem_v, void* ws, cudaStream_t st) {
-  const Shape sh = plan(a);
+  const Shape sh = plan(a, false);
   const Layout L = layout(a, sh);
   AttnParams P{};
   char* w = reinterpret_cast<char*>(ws);
@@ -912,3 +925,12 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
 }
 
 }  // namespace msa
+
+// Selects the attention kernel of later msa_attend calls in this process:
+// 0 = automatic, 1 = split-K, 2 = tensor cores (any row count); returns the
+// previous setting. A testing and benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_attend_kernel(int which) {
+  const int old = msa::g_attend_kernel;
+  if (which >= 0 && which <= 2) msa::g_attend_kernel = which;
+  return old;
+}

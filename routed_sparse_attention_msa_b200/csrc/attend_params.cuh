@@ -1,0 +1,51 @@
+// Parameter block shared by the attention kernels (split-K decoding in
+// attend.cu, the tensor-core kernel for many query rows in attend_tc.cu), and
+// the host-side hooks between them.
+#pragma once
+
+#include "msa_internal.cuh"
+
+namespace msa {
+
+struct AttnParams {
+  const uint16_t* q;
+  const uint16_t* k_loc;
+  const uint16_t* v_loc;
+  const uint16_t* mem_k;
+  const uint16_t* mem_v;
+  const int64_t* sel_off;
+  const int64_t* sel_chunk;
+  float* qrot;      // [n_q, hq, d]
+  float* krot;      // [n_loc, hkv, d]
+  float* part_o;    // [n_q, hq, splits, d]
+  float2* part_ml;  // [n_q, hq, splits]
+  unsigned* tickets;  // [n_tiles * hkv]
+  uint16_t* out;
+  float* out_f32;
+  float* lse;
+  int n_seq, n_q, n_loc, hq, hkv, group, rt, n_splits, n_tiles;
+  float scale;
+  double pos_offset, log2_theta;
+  int32_t q_seq_off[kMaxSeq + 1];
+  int32_t q_start[kMaxSeq];
+  int32_t loc_off[kMaxSeq + 1];
+  int32_t tile_off[kMaxSeq + 1];
+};
+
+// Index of the segment of `off` (n_seq + 1 ascending offsets) holding x.
+__device__ __forceinline__ int seq_of(const int32_t* off, int n_seq, int x) {
+  int lo = 0, hi = n_seq - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// attend_tc.cu: one CTA per (tile of 128 query vectors = rt rows x group q
+// heads, kv head); grid (n_tiles, hkv). Needs rope_rows to have run.
+constexpr int kAttnTcVec = 128;
+msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st);
+int attend_tc_error_take();  // 1 if its bounded wait ran out since the last call
+
+}  // namespace msa

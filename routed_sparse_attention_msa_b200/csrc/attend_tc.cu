@@ -1,0 +1,475 @@
+// Sparse attention for many query rows per sequence (prefill), on the tensor
+// cores.
+//
+// ["MSA: Memory Sparse Attention", Overall Design: Architecture — the selected
+// documents' compressed K/V are concatenated with the query's local K/V;
+// Parallel (document-wise) RoPE and Global RoPE offset by k (Figure 2)]
+//
+// Same result as the split-K kernel in attend.cu (which stays the decoding
+// path): every query row attends over its sequence's selected pooled K/V and
+// its local K/V up to its own position, GQA, softmax in fp32. With tens of
+// rows per sequence the logits and P.V are dense contractions, so here a CTA
+// owns 128 query vectors (rt rows x the GQA group's q heads) of one kv head
+// and walks the key list in blocks of 64:
+//   S = Q K^T     tcgen05 M128 x N64 x K128 into TMEM,
+//   softmax       one thread per query vector (its TMEM lane): running max
+//                 and sum in fp32, the block's P rounded to bf16 into shared
+//                 memory,
+// When (tiles x kv heads) would not fill the GPU, the key blocks are split
+// across CTAs, each writing an unnormalised partial that the last one to
+// finish merges by log-sum-exp.
+//   O += P V      tcgen05 M128 x N128 x K64, accumulated in TMEM across
+//                 blocks (P is taken against a reference max that moves only
+//                 when the running max passes it by more than 8; then the
+//                 thread rescales its O row in TMEM).
+// The rotated queries and local keys are fp32; each is split into a bf16 high
+// part and the bf16 rounding of the remainder, and S sums Qhi Khi + Qlo Khi +
+// Qhi Klo (the Qlo Klo term is below 2^-16 of the product), so the logits keep
+// fp32 accuracy. The pooled memory keys are bf16 already (exact). V is staged
+// transposed, so every operand is K-major with the 128-byte swizzle.
+// Every mbarrier wait is bounded in time, and every warp is reconverged
+// (__all_sync) after it: lanes leave a polling loop on different iterations,
+// and a diverged warp would run the softmax lane group by lane group.
+#include <cuda.h>
+
+#include "attend_params.cuh"
+#include "tc_ptx.cuh"
+
+namespace msa {
+namespace {
+
+using namespace tc;
+
+constexpr int kVec = kAttnTcVec;  // query vectors per CTA = TMEM lanes
+constexpr int kNK = 64;           // keys per block
+constexpr int kThreadsTc = 128;
+constexpr int kQAtom = kVec * 128;  // 16 KB: 128 rows x 64 dims (bf16)
+constexpr int kKAtom = kNK * 128;   // 8 KB: 64 keys x 64 dims
+constexpr int offQhi = 0;
+constexpr int offQlo = offQhi + 2 * kQAtom;
+constexpr int offKhi = offQlo + 2 * kQAtom;
+constexpr int offKlo = offKhi + 2 * kKAtom;
+constexpr int offVT = offKlo + 2 * kKAtom;  // 128 dims x 64 keys
+constexpr int offP = offVT + 128 * 128;     // 128 vectors x 64 keys
+constexpr int offIdx = offP + kVec * 128;  // 64 bank-row indices
+constexpr int offBar = offIdx + kNK * 8;
+constexpr int kSmemTc = 1024 + offBar + 64;
+constexpr int kTmemCols = 256;  // S: columns 0..63, O block: 128..255
+// instruction descriptors: D fp32, A/B bf16, K-major; M = 128; N = 64 or 128
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNK >> 3) << 17) | (8u << 24);
+constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) | (8u << 24);
+
+// 16-byte piece c (0..7) of row r of a 128-byte-swizzled K-major atom.
+__device__ __forceinline__ uint8_t* swz(uint8_t* atom, int r, int c) { return atom + r * 128 + ((c ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ float bf_round(float x) { return __uint_as_float(f2bf_bits(x) << 16); }
+
+// Eight fp32 values -> 16-byte bf16 high part and 16-byte bf16 remainder.
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = bf_round(x[i]);
+    l[i] = x[i] - h[i];
+  }
+  hi = make_uint4(pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]), pack_bf2(h[6], h[7]));
+  lo = make_uint4(pack_bf2(l[0], l[1]), pack_bf2(l[2], l[3]), pack_bf2(l[4], l[5]), pack_bf2(l[6], l[7]));
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int64_t* s_idx = reinterpret_cast<int64_t*>(smem + offIdx);  // bank rows of this block's memory keys
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + offBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tile = blockIdx.x, kvh = blockIdx.y, sp_idx = blockIdx.z;
+  const int s = seq_of(p.tile_off, p.n_seq, tile);
+  const int row0 = p.q_seq_off[s] + (tile - p.tile_off[s]) * p.rt;
+  const int nr = min(p.rt, p.q_seq_off[s + 1] - row0);
+  const int g0 = p.q_start[s] + (row0 - p.q_seq_off[s]);  // active index of the tile's first row
+  const int n_loc_s = p.loc_off[s + 1] - p.loc_off[s];
+  const int lvis = max(0, min(n_loc_s, g0 + nr));  // local keys visible to the last row
+  const size_t row_stride = (size_t)p.hkv * kHeadDim;
+
+  // this thread's query vector: row rr of the tile, q head gg of the group
+  const int rr = tid / p.group, gg = tid % p.group;
+  const bool vvalid = rr < nr;
+  const int gv = vvalid ? g0 + rr : -1;
+
+  if (tid == 0) {
+    mbar_init(smem_u32(bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  pdl_wait();  // the rotated rows and the selection come from earlier kernels
+  pdl_trigger();
+  const int64_t mem_base = __ldg(p.sel_off + s);
+  const int64_t n_mem = __ldg(p.sel_off + s + 1) - mem_base;
+  const int64_t n_keys = n_mem + lvis;
+  // this CTA's share of the key blocks (split-K when the grid is small)
+  const int64_t n_blocks = (n_keys + kNK - 1) / kNK;
+  const int64_t per = (n_blocks + p.n_splits - 1) / p.n_splits;
+  const int64_t k_begin = min(n_keys, (int64_t)sp_idx * per * kNK);
+  const int64_t k_end = min(n_keys, k_begin + per * kNK);
+
+  {  // Q (high and low parts), this thread's row, both 64-dimension atoms, 4 pieces per round
+    const float4* qv = reinterpret_cast<const float4*>(
+        p.qrot + ((size_t)(row0 + (vvalid ? rr : 0)) * p.hq + kvh * p.group + gg) * kHeadDim);
+#pragma unroll
+    for (int c0 = 0; c0 < 16; c0 += 4) {
+      float4 x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = vvalid ? __ldg(qv + 2 * c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u;
+        const float f[8] = {x[2 * u].x, x[2 * u].y, x[2 * u].z, x[2 * u].w,
+                            x[2 * u + 1].x, x[2 * u + 1].y, x[2 * u + 1].z, x[2 * u + 1].w};
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        *reinterpret_cast<uint4*>(swz(smem + offQhi + (c >> 3) * kQAtom, tid, c & 7)) = hi;
+        *reinterpret_cast<uint4*>(swz(smem + offQlo + (c >> 3) * kQAtom, tid, c & 7)) = lo;
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t tmem_o = tmem + 128;
+
+  // Softmax state of this thread's vector. P is taken relative to m_ref, which
+  // moves only when the running max exceeds it by more than 8 (then the
+  // thread's O row in TMEM is rescaled), so P <= e^8 and P.V accumulates in
+  // TMEM across blocks.
+  float m_ref = -INFINITY, l = 0.f;
+  uint32_t phase = 0;
+  bool ok = true, pv_pending = false;
+  int blk = 0;
+
+  for (int64_t kb = k_begin; kb < k_end; kb += kNK, ++blk) {
+    const int nb = (int)min((int64_t)kNK, k_end - kb);
+    const bool has_local = kb + nb > n_mem;
+    if (pv_pending) {  // the previous block's P.V still reads V^T and P
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
+      phase ^= 1;
+      pv_pending = false;
+      if (!__syncthreads_and(ok)) { ok = false; break; }
+      tc_fence_after();
+    }
+    if (tid < nb && kb + tid < n_mem)
+      s_idx[tid] = p.sel_chunk ? __ldg(p.sel_chunk + mem_base + kb + tid) : mem_base + kb + tid;
+    __syncthreads();
+
+    // ---- K (high, low): 64 keys x 16 pieces of 8 dims, 8 pieces per thread in two rounds
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint4 raw[4];
+      float4 fa[4], fb[4];
+      int kind[4];  // 0 none, 1 memory, 2 local
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = tid + (4 * half + u) * kThreadsTc;
+        const int jj = idx >> 4, c = idx & 15;
+        const int64_t key = kb + jj;
+        kind[u] = jj >= nb ? 0 : key < n_mem ? 1 : 2;
+        raw[u] = make_uint4(0, 0, 0, 0);
+        fa[u] = fb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kind[u] == 1) {
+          raw[u] = __ldg(reinterpret_cast<const uint4*>(p.mem_k + (size_t)s_idx[jj] * row_stride +
+                                                        (size_t)kvh * kHeadDim + 8 * c));
+        } else if (kind[u] == 2) {
+          const float4* kr = reinterpret_cast<const float4*>(
+              p.krot + ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim);
+          fa[u] = __ldg(kr + 2 * c);
+          fb[u] = __ldg(kr + 2 * c + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = tid + (4 * half + u) * kThreadsTc;
+        const int jj = idx >> 4, c = idx & 15;
+        uint4 hi = raw[u], lo = make_uint4(0, 0, 0, 0);
+        if (kind[u] == 2) {
+          const float f[8] = {fa[u].x, fa[u].y, fa[u].z, fa[u].w, fb[u].x, fb[u].y, fb[u].z, fb[u].w};
+          split8(f, hi, lo);
+        }
+        *reinterpret_cast<uint4*>(swz(smem + offKhi + (c >> 3) * kKAtom, jj, c & 7)) = hi;
+        if (has_local) *reinterpret_cast<uint4*>(swz(smem + offKlo + (c >> 3) * kKAtom, jj, c & 7)) = lo;
+      }
+    }
+    {  // V^T: this thread takes keys 2 jp, 2 jp + 1 and dimensions 32 dg .. 32 dg + 31
+      const int jp = tid & 31, dg = tid >> 5;
+      uint4 x[2][4];
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int jj = 2 * jp + k2;
+        const int64_t key = kb + jj;
+        const uint16_t* vr = nullptr;
+        if (jj < nb && key < n_mem)
+          vr = p.mem_v + (size_t)s_idx[jj] * row_stride + (size_t)kvh * kHeadDim;
+        else if (jj < nb)
+          vr = p.v_loc + ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          x[k2][i] = vr ? __ldg(reinterpret_cast<const uint4*>(vr + 32 * dg) + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int d = 0; d < 32; ++d) {
+        const uint4& a = x[0][d >> 3];
+        const uint4& b = x[1][d >> 3];
+        const int w = (d >> 1) & 3;
+        const uint32_t wa = w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
+        const uint32_t wb = w == 0 ? b.x : w == 1 ? b.y : w == 2 ? b.z : b.w;
+        const int dim = 32 * dg + d;
+        *reinterpret_cast<uint32_t*>(swz(smem + offVT, dim, jp >> 2) + 4 * (jp & 3)) =
+            __byte_perm(wa, wb, (d & 1) ? 0x7632 : 0x5410);
+      }
+    }
+    fence_proxy_async_smem();  // the MMAs read these bytes through the async proxy
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- S = Q K^T
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t qa = (uint32_t)((k >> 2) * kQAtom + (k & 3) * 32);
+        const uint32_t ko = (uint32_t)((k >> 2) * kKAtom + (k & 3) * 32);
+        const uint64_t dkhi = sw128_desc(smem_u32(smem + offKhi) + ko);
+        tc_mma(tmem, sw128_desc(smem_u32(smem + offQhi) + qa), dkhi, kIdescS, k > 0 ? 1u : 0u);
+        tc_mma(tmem, sw128_desc(smem_u32(smem + offQlo) + qa), dkhi, kIdescS, 1u);
+        if (has_local)
+          tc_mma(tmem, sw128_desc(smem_u32(smem + offQhi) + qa), sw128_desc(smem_u32(smem + offKlo) + ko), kIdescS,
+                 1u);
+      }
+      tc_commit(smem_u32(bar));
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
+    phase ^= 1;
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc_fence_after();
+
+    // ---- softmax of this thread's vector against the block
+    float sv[kNK];
+    tmem_ld32(tmem + lane_base, sv);
+    tmem_ld32(tmem + lane_base + 32, sv + 32);
+    tmem_ld_wait();
+    // Logits in log2 units (scale * log2 e) so that P = 2^(s - m_ref). Key j
+    // of the block is visible to this vector iff j < jvis: the block's
+    // memory keys always, its local keys up to the row's own position.
+    const int jmem = (int)max((int64_t)0, min((int64_t)nb, n_mem - kb));  // memory keys in the block
+    const int jloc = (int)(gv - max((int64_t)0, kb - n_mem)) + 1;         // local keys it sees
+    const int jvis = !vvalid ? 0 : min(nb, jmem + max(0, min(nb - jmem, jloc)));
+    const float sl2 = p.scale * 1.4426950408889634f;
+    float bm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kNK; ++j) {
+      sv[j] = j < jvis ? sv[j] * sl2 : -INFINITY;
+      bm = fmaxf(bm, sv[j]);
+    }
+    const bool move = bm > m_ref + 11.5f;  // 2^11.5 ~ e^8; also when m_ref is -inf and bm finite
+    const float corr = !move ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - bm));
+    if (move) m_ref = bm;
+    const float mr = m_ref == -INFINITY ? 0.f : m_ref;  // all P are 0 then (2^-inf)
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float pr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        pr[i] = exp2f(sv[8 * c + i] - mr);
+        sum += pr[i];
+      }
+      *reinterpret_cast<uint4*>(swz(smem + offP, tid, c)) =
+          make_uint4(pack_bf2(pr[0], pr[1]), pack_bf2(pr[2], pr[3]), pack_bf2(pr[4], pr[5]), pack_bf2(pr[6], pr[7]));
+    }
+    l = l * corr + sum;
+    // rescale this warp's O rows in TMEM when any of its lanes moved its reference
+    if (blk > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+      for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+        float t[16];
+        tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) t[j] *= corr;
+        tmem_st16(tmem_o + lane_base + 16 * cc, t);
+      }
+      tmem_st_wait();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- O += P V (accumulated in TMEM; waited for before V^T and P are reused)
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < kNK / 16; ++k)
+        tc_mma(tmem_o, sw128_desc(smem_u32(smem + offP) + k * 32), sw128_desc(smem_u32(smem + offVT) + k * 32),
+               kIdescO, (blk > 0 || k > 0) ? 1u : 0u);
+      tc_commit(smem_u32(bar));
+    }
+    pv_pending = true;
+  }
+  if (ok && pv_pending) {
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
+    phase ^= 1;
+    ok = __syncthreads_and(ok);
+  }
+  if (!ok && tid == 0) {  // a wait ran out: let the MMAs in flight finish (bounded) before TMEM is freed
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try(smem_u32(bar), phase ^ 1) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+  tc_fence_after();
+
+  // ---- split-K: unnormalised partial (o, m, l) out; the last CTA of the
+  // (tile, kv head) merges by log-sum-exp
+  if (p.n_splits > 1) {
+    __shared__ int s_last;
+    const int row = row0 + rr, h = kvh * p.group + gg;
+    const size_t pi = ((size_t)row * p.hq + h) * p.n_splits + sp_idx;
+    if (ok) {
+#pragma unroll 1
+      for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+        float t[16];
+        if (blk > 0) {
+          tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) t[j] = 0.f;
+        }
+        if (vvalid) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + pi * kHeadDim + 16 * cc);
+          dst[0] = make_float4(t[0], t[1], t[2], t[3]);
+          dst[1] = make_float4(t[4], t[5], t[6], t[7]);
+          dst[2] = make_float4(t[8], t[9], t[10], t[11]);
+          dst[3] = make_float4(t[12], t[13], t[14], t[15]);
+        }
+      }
+      if (vvalid) p.part_ml[pi] = make_float2(m_ref, l);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(p.tickets + (size_t)tile * p.hkv + kvh, 1u) == (unsigned)(p.n_splits - 1);
+    __syncthreads();
+    if (s_last && vvalid) {
+      __threadfence();
+      const size_t rh = (size_t)row * p.hq + h;
+      float mm = -INFINITY;
+      for (int j = 0; j < p.n_splits; ++j) {
+        const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
+        if (x.y > 0.f) mm = fmaxf(mm, x.x);
+      }
+      float wsum = 0.f;
+      for (int j = 0; j < p.n_splits; ++j) {
+        const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
+        if (x.y > 0.f) wsum += x.y * exp2f(x.x - mm);
+      }
+      const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+      const size_t base = rh * kHeadDim;
+#pragma unroll 4  // several dimension chunks' loads in flight
+      for (int d = 0; d < kHeadDim; d += 8) {
+        float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < p.n_splits; ++j) {
+          const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
+          if (!(x.y > 0.f)) continue;
+          const float w = exp2f(x.x - mm);
+          const float4* src = reinterpret_cast<const float4*>(p.part_o + (rh * p.n_splits + j) * kHeadDim + d);
+          const float4 a = __ldcg(src), b = __ldcg(src + 1);
+          r[0] += w * a.x; r[1] += w * a.y; r[2] += w * a.z; r[3] += w * a.w;
+          r[4] += w * b.x; r[5] += w * b.y; r[6] += w * b.z; r[7] += w * b.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] *= inv;
+        *reinterpret_cast<uint4*>(p.out + base + d) =
+            make_uint4(pack_bf2(r[0], r[1]), pack_bf2(r[2], r[3]), pack_bf2(r[4], r[5]), pack_bf2(r[6], r[7]));
+        if (p.out_f32) {
+          reinterpret_cast<float4*>(p.out_f32 + base + d)[0] = make_float4(r[0], r[1], r[2], r[3]);
+          reinterpret_cast<float4*>(p.out_f32 + base + d)[1] = make_float4(r[4], r[5], r[6], r[7]);
+        }
+      }
+      if (p.lse) p.lse[rh] = wsum > 0.f ? (mm + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+    }
+  } else if (ok) {  // ---- one CTA per (tile, kv head): normalised output, log-sum-exp
+    const int row = row0 + rr, h = kvh * p.group + gg;
+    const float inv = l > 0.f ? 1.0f / l : 0.f;
+    const size_t base = ((size_t)row * p.hq + h) * kHeadDim;
+#pragma unroll 1
+    for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+      float t[16];
+      if (blk > 0) {  // warp-uniform: every lane of the CTA walked the same blocks
+        tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) t[j] = 0.f;
+      }
+      if (vvalid) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 8) {
+          float r[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) r[i] = t[j + i] * inv;
+          *reinterpret_cast<uint4*>(p.out + base + 16 * cc + j) =
+              make_uint4(pack_bf2(r[0], r[1]), pack_bf2(r[2], r[3]), pack_bf2(r[4], r[5]), pack_bf2(r[6], r[7]));
+          if (p.out_f32) {
+            reinterpret_cast<float4*>(p.out_f32 + base + 16 * cc + j)[0] = make_float4(r[0], r[1], r[2], r[3]);
+            reinterpret_cast<float4*>(p.out_f32 + base + 16 * cc + j)[1] = make_float4(r[4], r[5], r[6], r[7]);
+          }
+        }
+      }
+    }
+    if (vvalid && p.lse)  // m_ref and l are in log2 units
+      p.lse[(size_t)row * p.hq + h] = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTmemCols));
+  }
+}
+
+}  // namespace
+
+msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
+    if (e != cudaSuccess) return cuda_fail(e, "attend: tensor-core kernel shared memory");
+    attr = true;
+  }
+  cudaError_t e = launch_pdl(attend_tc_kernel, dim3((unsigned)P.n_tiles, (unsigned)P.hkv, (unsigned)P.n_splits),
+                             dim3(kThreadsTc),
+                             (size_t)kSmemTc, st, P);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: tensor cores (many rows)");
+  return launch_check("attend: tensor cores (many rows)");
+}
+
+int attend_tc_error_take() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof v) != cudaSuccess) return 0;
+  if (v) {
+    int z = 0;
+    cudaMemcpyToSymbol(g_tc_error, &z, sizeof z);
+  }
+  return v;
+}
+
+}  // namespace msa

@@ -303,7 +303,9 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < C::kCols; ++j) acc[j] = 0.f;
         for (int h = 0; h < kHeads; ++h) {
-          if (!mbar_wait(smem_u32(&tfull[b]), tph, abort_flag)) { ok = false; break; }
+          // __all_sync: the lanes leave the wait on different polls; the warp
+          // must be converged again for the aligned TMEM loads and the math.
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[b]), tph, abort_flag))) { ok = false; break; }
           tc_fence_after();
           const float kh = s_ik[h * 32 + lane];
           const float2 k2 = make_float2(kh, kh);

@@ -256,7 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int nb = 0; nb < a.n_nb; ++nb, ++blk) {
         const int b = blk & 1;
         if (a.n_nb > 1) load_block(nb * NB);
-        if (!mbar_wait(smem_u32(&tfull[b]), (blk >> 1) & 1, abort_flag)) { ok = false; break; }
+        // __all_sync: the lanes leave the wait on different polls; the warp
+        // must be converged again for the aligned TMEM loads and the math.
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[b]), (blk >> 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
         // Stream over the block's columns: the score of (row, column), a
         // running max over the current sequence's columns, and a flush (warp

@@ -264,6 +264,13 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
+@pytest.fixture(params=["split", "tc"])
+def attend_kernel(request, msa):
+    old = msa.set_attend_kernel(request.param)
+    yield request.param
+    msa.set_attend_kernel(old)
+
+
 def _attend_case(rows, n_loc, n_mem, q_start, C=3000, hq=32, hkv=8, layer=20):
     T, L = sum(rows), sum(n_loc)
     q = host_normal((T, hq, 128), synth.tid("q_att", layer))
@@ -308,8 +315,13 @@ def _attend_gpu(msa, c, pos_offset, theta=1e6, identity=False):
     dict(rows=(1,), n_loc=(129,), n_mem=(1500,), q_start=(128,)),                # many keys: split-K
     dict(rows=(1, 1, 1), n_loc=(65, 1, 7), n_mem=(0, 300, 61), q_start=(64, 0, 6)),  # empty memory
     dict(rows=(5,), n_loc=(3,), n_mem=(9,), q_start=(0,)),                       # rows beyond local keys
+    dict(rows=(64, 64, 30), n_loc=(64, 64, 30), n_mem=(250, 130, 0), q_start=(0, 0, 0)),  # prefill, 3 sequences
+    dict(rows=(48,), n_loc=(80,), n_mem=(100,), q_start=(32,)),                  # prefill after a local prefix
+    dict(rows=(100,), n_loc=(100,), n_mem=(77,), q_start=(0,), hq=8, hkv=8),    # no GQA sharing (group 1)
+    dict(rows=(40, 9), n_loc=(40, 9), n_mem=(64, 200), q_start=(0, 0), hq=64, hkv=8),  # group 8
+    dict(rows=(32,) * 19, n_loc=(32,) * 19, n_mem=(40,) * 19, q_start=(0,) * 19),  # >= 148 CTAs: no key split
 ])
-def test_attend_matches_oracle(msa, case):
+def test_attend_matches_oracle(msa, attend_kernel, case):
     c = _attend_case(**case)
     pos = 16.0
     g_out, g_f32, g_lse = _attend_gpu(msa, c, pos)
@@ -320,7 +332,7 @@ def test_attend_matches_oracle(msa, case):
     np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
 
 
-def test_attend_block_length_offset_reading(msa):
+def test_attend_block_length_offset_reading(msa, attend_kernel):
     """The alternative reading of the query offset: k retrieved documents x the
     chunk length (pos_offset = 16 * 64) instead of k."""
     c = _attend_case(rows=(2, 1), n_loc=(5, 70), n_mem=(48, 90), q_start=(3, 69), layer=22)
@@ -330,7 +342,7 @@ def test_attend_block_length_offset_reading(msa):
     np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
 
 
-def test_attend_staged_memory_equals_indexed(msa):
+def test_attend_staged_memory_equals_indexed(msa, attend_kernel):
     c = _attend_case(rows=(2, 1), n_loc=(4, 9), n_mem=(33, 70), q_start=(2, 8), layer=21)
     a = _attend_gpu(msa, c, 16.0)
     b = _attend_gpu(msa, c, 16.0, identity=True)
