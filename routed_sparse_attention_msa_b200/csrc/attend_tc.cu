@@ -12,16 +12,17 @@
 // owns 128 query vectors (rt rows x the GQA group's q heads) of one kv head
 // and walks the key list in blocks of 64:
 //   S = Q K^T     tcgen05 M128 x N64 x K128 into TMEM,
-//   softmax       one thread per query vector (its TMEM lane): running max
-//                 and sum in fp32, the block's P rounded to bf16 into shared
-//                 memory,
+//   softmax       two threads per query vector (its TMEM lane; one per 32-key
+//                 half of the block, exchanging the block max through shared
+//                 memory): running max and sum in fp32, the block's P
+//                 rounded to bf16 into shared memory,
 // When (tiles x kv heads) would not fill the GPU, the key blocks are split
 // across CTAs, each writing an unnormalised partial that the last one to
 // finish merges by log-sum-exp.
 //   O += P V      tcgen05 M128 x N128 x K64, accumulated in TMEM across
 //                 blocks (P is taken against a reference max that moves only
-//                 when the running max passes it by more than 8; then the
-//                 thread rescales its O row in TMEM).
+//                 when the running max passes it by more than 2^11.5; then
+//                 the two threads rescale their halves of the O row in TMEM).
 // The rotated queries and local keys are fp32; each is split into a bf16 high
 // part and the bf16 rounding of the remainder, and S sums Qhi Khi + Qlo Khi +
 // Qhi Klo (the Qlo Klo term is below 2^-16 of the product), so the logits keep
@@ -42,7 +43,7 @@ using namespace tc;
 
 constexpr int kVec = kAttnTcVec;  // query vectors per CTA = TMEM lanes
 constexpr int kNK = 64;           // keys per block
-constexpr int kThreadsTc = 128;
+constexpr int kThreadsTc = 256;  // 8 warps: (lane quadrant, half) pairs
 constexpr int kQAtom = kVec * 128;  // 16 KB: 128 rows x 64 dims (bf16)
 constexpr int kKAtom = kNK * 128;   // 8 KB: 64 keys x 64 dims
 constexpr int offQhi = 0;
@@ -52,7 +53,8 @@ constexpr int offKlo = offKhi + 2 * kKAtom;
 constexpr int offVT = offKlo + 2 * kKAtom;  // 128 dims x 64 keys
 constexpr int offP = offVT + 128 * 128;     // 128 vectors x 64 keys
 constexpr int offIdx = offP + kVec * 128;  // 64 bank-row indices
-constexpr int offBar = offIdx + kNK * 8;
+constexpr int offMax = offIdx + kNK * 8;   // [2][128] block maxima, then the two partial sums
+constexpr int offBar = offMax + 2 * kVec * 4;
 constexpr int kSmemTc = 1024 + offBar + 64;
 constexpr int kTmemCols = 256;  // S: columns 0..63, O block: 128..255
 // instruction descriptors: D fp32, A/B bf16, K-major; M = 128; N = 64 or 128
@@ -80,11 +82,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int64_t* s_idx = reinterpret_cast<int64_t*>(smem + offIdx);  // bank rows of this block's memory keys
+  float* s_max = reinterpret_cast<float*>(smem + offMax);      // [half][vector]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + offBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q = warp & 3, hs = warp >> 2;  // TMEM lane quadrant; which half of keys / dimensions
+  const int v = 32 * q + lane;             // this thread's query vector (TMEM lane)
   const int tile = blockIdx.x, kvh = blockIdx.y, sp_idx = blockIdx.z;
   const int s = seq_of(p.tile_off, p.n_seq, tile);
   const int row0 = p.q_seq_off[s] + (tile - p.tile_off[s]) * p.rt;
@@ -94,8 +99,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   const int lvis = max(0, min(n_loc_s, g0 + nr));  // local keys visible to the last row
   const size_t row_stride = (size_t)p.hkv * kHeadDim;
 
-  // this thread's query vector: row rr of the tile, q head gg of the group
-  const int rr = tid / p.group, gg = tid % p.group;
+  // the query vector: row rr of the tile, q head gg of the group
+  const int rr = v / p.group, gg = v % p.group;
   const bool vvalid = rr < nr;
   const int gv = vvalid ? g0 + rr : -1;
 
@@ -120,11 +125,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   const int64_t k_begin = min(n_keys, (int64_t)sp_idx * per * kNK);
   const int64_t k_end = min(n_keys, k_begin + per * kNK);
 
-  {  // Q (high and low parts), this thread's row, both 64-dimension atoms, 4 pieces per round
+  {  // Q (high and low parts): this thread stages its vector's 64-dimension atom hs
     const float4* qv = reinterpret_cast<const float4*>(
-        p.qrot + ((size_t)(row0 + (vvalid ? rr : 0)) * p.hq + kvh * p.group + gg) * kHeadDim);
+        p.qrot + ((size_t)(row0 + (vvalid ? rr : 0)) * p.hq + kvh * p.group + gg) * kHeadDim + 64 * hs);
 #pragma unroll
-    for (int c0 = 0; c0 < 16; c0 += 4) {
+    for (int c0 = 0; c0 < 8; c0 += 4) {
       float4 x[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = vvalid ? __ldg(qv + 2 * c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -135,8 +140,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
                             x[2 * u + 1].x, x[2 * u + 1].y, x[2 * u + 1].z, x[2 * u + 1].w};
         uint4 hi, lo;
         split8(f, hi, lo);
-        *reinterpret_cast<uint4*>(swz(smem + offQhi + (c >> 3) * kQAtom, tid, c & 7)) = hi;
-        *reinterpret_cast<uint4*>(swz(smem + offQlo + (c >> 3) * kQAtom, tid, c & 7)) = lo;
+        *reinterpret_cast<uint4*>(swz(smem + offQhi + hs * kQAtom, v, c)) = hi;
+        *reinterpret_cast<uint4*>(swz(smem + offQlo + hs * kQAtom, v, c)) = lo;
       }
     }
   }
@@ -145,14 +150,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_base = (uint32_t)(32 * q) << 16;
   const uint32_t tmem_o = tmem + 128;
 
-  // Softmax state of this thread's vector. P is taken relative to m_ref, which
-  // moves only when the running max exceeds it by more than 8 (then the
-  // thread's O row in TMEM is rescaled), so P <= e^8 and P.V accumulates in
-  // TMEM across blocks.
-  float m_ref = -INFINITY, l = 0.f;
+  // Softmax state of the vector (identical in both of its threads). P is
+  // taken relative to m_ref (log2 units), which moves only when the running
+  // max exceeds it by more than 11.5 (then both threads rescale their halves
+  // of the O row in TMEM), so P <= 2^11.5 and P.V accumulates in TMEM across
+  // blocks. l_own sums this thread's keys only; the halves add at the end.
+  float m_ref = -INFINITY, l_own = 0.f;
   uint32_t phase = 0;
   bool ok = true, pv_pending = false;
   int blk = 0;
@@ -171,15 +177,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
       s_idx[tid] = p.sel_chunk ? __ldg(p.sel_chunk + mem_base + kb + tid) : mem_base + kb + tid;
     __syncthreads();
 
-    // ---- K (high, low): 64 keys x 16 pieces of 8 dims, 8 pieces per thread in two rounds
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    {  // ---- K (high, low): 64 keys x 16 pieces of 8 dims, 4 pieces per thread
       uint4 raw[4];
       float4 fa[4], fb[4];
       int kind[4];  // 0 none, 1 memory, 2 local
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int idx = tid + (4 * half + u) * kThreadsTc;
+        const int idx = tid + u * kThreadsTc;
         const int jj = idx >> 4, c = idx & 15;
         const int64_t key = kb + jj;
         kind[u] = jj >= nb ? 0 : key < n_mem ? 1 : 2;
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int idx = tid + (4 * half + u) * kThreadsTc;
+        const int idx = tid + u * kThreadsTc;
         const int jj = idx >> 4, c = idx & 15;
         uint4 hi = raw[u], lo = make_uint4(0, 0, 0, 0);
         if (kind[u] == 2) {
@@ -208,9 +212,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
         if (has_local) *reinterpret_cast<uint4*>(swz(smem + offKlo + (c >> 3) * kKAtom, jj, c & 7)) = lo;
       }
     }
-    {  // V^T: this thread takes keys 2 jp, 2 jp + 1 and dimensions 32 dg .. 32 dg + 31
+    {  // V^T: this thread takes keys 2 jp, 2 jp + 1 and dimensions 16 dg .. 16 dg + 15
       const int jp = tid & 31, dg = tid >> 5;
-      uint4 x[2][4];
+      uint4 x[2][2];
 #pragma unroll
       for (int k2 = 0; k2 < 2; ++k2) {
         const int jj = 2 * jp + k2;
@@ -221,17 +225,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
         else if (jj < nb)
           vr = p.v_loc + ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          x[k2][i] = vr ? __ldg(reinterpret_cast<const uint4*>(vr + 32 * dg) + i) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 2; ++i)
+          x[k2][i] = vr ? __ldg(reinterpret_cast<const uint4*>(vr + 16 * dg) + i) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int d = 0; d < 32; ++d) {
+      for (int d = 0; d < 16; ++d) {
         const uint4& a = x[0][d >> 3];
         const uint4& b = x[1][d >> 3];
         const int w = (d >> 1) & 3;
         const uint32_t wa = w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
         const uint32_t wb = w == 0 ? b.x : w == 1 ? b.y : w == 2 ? b.z : b.w;
-        const int dim = 32 * dg + d;
+        const int dim = 16 * dg + d;
         *reinterpret_cast<uint32_t*>(swz(smem + offVT, dim, jp >> 2) + 4 * (jp & 3)) =
             __byte_perm(wa, wb, (d & 1) ? 0x7632 : 0x5410);
       }
@@ -261,51 +265,53 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc_fence_after();
 
-    // ---- softmax of this thread's vector against the block
-    float sv[kNK];
-    tmem_ld32(tmem + lane_base, sv);
-    tmem_ld32(tmem + lane_base + 32, sv + 32);
+    // ---- softmax: this thread's 32 keys (32 hs .. 32 hs + 31) of its vector
+    float sv[32];
+    tmem_ld32(tmem + lane_base + 32 * hs, sv);
     tmem_ld_wait();
     // Logits in log2 units (scale * log2 e) so that P = 2^(s - m_ref). Key j
-    // of the block is visible to this vector iff j < jvis: the block's
-    // memory keys always, its local keys up to the row's own position.
+    // of the block is visible to this vector iff j < jvis: the block's memory
+    // keys always, its local keys up to the row's own position.
     const int jmem = (int)max((int64_t)0, min((int64_t)nb, n_mem - kb));  // memory keys in the block
     const int jloc = (int)(gv - max((int64_t)0, kb - n_mem)) + 1;         // local keys it sees
-    const int jvis = !vvalid ? 0 : min(nb, jmem + max(0, min(nb - jmem, jloc)));
+    const int jvis = (!vvalid ? 0 : min(nb, jmem + max(0, min(nb - jmem, jloc)))) - 32 * hs;
     const float sl2 = p.scale * 1.4426950408889634f;
-    float bm = -INFINITY;
+    float bmo = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kNK; ++j) {
+    for (int j = 0; j < 32; ++j) {
       sv[j] = j < jvis ? sv[j] * sl2 : -INFINITY;
-      bm = fmaxf(bm, sv[j]);
+      bmo = fmaxf(bmo, sv[j]);
     }
+    s_max[hs * kVec + v] = bmo;
+    __syncthreads();
+    const float bm = fmaxf(s_max[v], s_max[kVec + v]);
     const bool move = bm > m_ref + 11.5f;  // 2^11.5 ~ e^8; also when m_ref is -inf and bm finite
     const float corr = !move ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - bm));
     if (move) m_ref = bm;
     const float mr = m_ref == -INFINITY ? 0.f : m_ref;  // all P are 0 then (2^-inf)
     float sum = 0.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       float pr[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         pr[i] = exp2f(sv[8 * c + i] - mr);
         sum += pr[i];
       }
-      *reinterpret_cast<uint4*>(swz(smem + offP, tid, c)) =
+      *reinterpret_cast<uint4*>(swz(smem + offP, v, 4 * hs + c)) =
           make_uint4(pack_bf2(pr[0], pr[1]), pack_bf2(pr[2], pr[3]), pack_bf2(pr[4], pr[5]), pack_bf2(pr[6], pr[7]));
     }
-    l = l * corr + sum;
-    // rescale this warp's O rows in TMEM when any of its lanes moved its reference
+    l_own = l_own * corr + sum;
+    // rescale this thread's half of the O row when any lane of the warp moved its reference
     if (blk > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll 1
-      for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         float t[16];
-        tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+        tmem_ld16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) t[j] *= corr;
-        tmem_st16(tmem_o + lane_base + 16 * cc, t);
+        tmem_st16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
       }
       tmem_st_wait();
     }
@@ -335,33 +341,38 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
     }
   }
   tc_fence_after();
+  // the vector's sum over both halves
+  s_max[hs * kVec + v] = l_own;
+  __syncthreads();
+  const float l = s_max[v] + s_max[kVec + v];
+  const int row = row0 + rr, h = kvh * p.group + gg;
+  const size_t rh = (size_t)row * p.hq + h;
 
-  // ---- split-K: unnormalised partial (o, m, l) out; the last CTA of the
-  // (tile, kv head) merges by log-sum-exp
   if (p.n_splits > 1) {
+    // ---- split-K: unnormalised partial (o, m, l) out; the last CTA of the
+    // (tile, kv head) merges by log-sum-exp
     __shared__ int s_last;
-    const int row = row0 + rr, h = kvh * p.group + gg;
-    const size_t pi = ((size_t)row * p.hq + h) * p.n_splits + sp_idx;
+    const size_t pi = rh * p.n_splits + sp_idx;
     if (ok) {
 #pragma unroll 1
-      for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         float t[16];
         if (blk > 0) {
-          tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+          tmem_ld16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
           tmem_ld_wait();
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) t[j] = 0.f;
         }
         if (vvalid) {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + pi * kHeadDim + 16 * cc);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + pi * kHeadDim + 64 * hs + 16 * cc);
           dst[0] = make_float4(t[0], t[1], t[2], t[3]);
           dst[1] = make_float4(t[4], t[5], t[6], t[7]);
           dst[2] = make_float4(t[8], t[9], t[10], t[11]);
           dst[3] = make_float4(t[12], t[13], t[14], t[15]);
         }
       }
-      if (vvalid) p.part_ml[pi] = make_float2(m_ref, l);
+      if (vvalid && hs == 0) p.part_ml[pi] = make_float2(m_ref, l);
     }
     __threadfence();
     __syncthreads();
@@ -369,7 +380,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
     __syncthreads();
     if (s_last && vvalid) {
       __threadfence();
-      const size_t rh = (size_t)row * p.hq + h;
       float mm = -INFINITY;
       for (int j = 0; j < p.n_splits; ++j) {
         const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
@@ -381,15 +391,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
         if (x.y > 0.f) wsum += x.y * exp2f(x.x - mm);
       }
       const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
-      const size_t base = rh * kHeadDim;
+      const size_t base = rh * kHeadDim + 64 * hs;
 #pragma unroll 4  // several dimension chunks' loads in flight
-      for (int d = 0; d < kHeadDim; d += 8) {
+      for (int d = 0; d < 64; d += 8) {
         float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < p.n_splits; ++j) {
           const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
           if (!(x.y > 0.f)) continue;
           const float w = exp2f(x.x - mm);
-          const float4* src = reinterpret_cast<const float4*>(p.part_o + (rh * p.n_splits + j) * kHeadDim + d);
+          const float4* src =
+              reinterpret_cast<const float4*>(p.part_o + (rh * p.n_splits + j) * kHeadDim + 64 * hs + d);
           const float4 a = __ldcg(src), b = __ldcg(src + 1);
           r[0] += w * a.x; r[1] += w * a.y; r[2] += w * a.z; r[3] += w * a.w;
           r[4] += w * b.x; r[5] += w * b.y; r[6] += w * b.z; r[7] += w * b.w;
@@ -403,17 +414,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
           reinterpret_cast<float4*>(p.out_f32 + base + d)[1] = make_float4(r[4], r[5], r[6], r[7]);
         }
       }
-      if (p.lse) p.lse[rh] = wsum > 0.f ? (mm + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+      if (p.lse && hs == 0) p.lse[rh] = wsum > 0.f ? (mm + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
     }
   } else if (ok) {  // ---- one CTA per (tile, kv head): normalised output, log-sum-exp
-    const int row = row0 + rr, h = kvh * p.group + gg;
     const float inv = l > 0.f ? 1.0f / l : 0.f;
-    const size_t base = ((size_t)row * p.hq + h) * kHeadDim;
+    const size_t base = rh * kHeadDim + 64 * hs;
 #pragma unroll 1
-    for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+    for (int cc = 0; cc < 4; ++cc) {
       float t[16];
-      if (blk > 0) {  // warp-uniform: every lane of the CTA walked the same blocks
-        tmem_ld16(tmem_o + lane_base + 16 * cc, t);
+      if (blk > 0) {  // uniform: every thread of the CTA walked the same blocks
+        tmem_ld16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
         tmem_ld_wait();
       } else {
 #pragma unroll
@@ -434,8 +444,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
         }
       }
     }
-    if (vvalid && p.lse)  // m_ref and l are in log2 units
-      p.lse[(size_t)row * p.hq + h] = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    if (vvalid && hs == 0 && p.lse)  // m_ref and l are in log2 units
+      p.lse[rh] = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
   }
 
   tc_fence_before();
