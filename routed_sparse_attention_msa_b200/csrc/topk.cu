@@ -9,7 +9,8 @@
 // and all keys are distinct. A document that was never scored (no chunks)
 // has score word 0, below every real score.
 //
-// k <= 16: each warp keeps its best 16 keys sorted across lanes 0..15. A batch
+// k <= 16: each warp keeps its best 16 keys sorted across lanes 0..15 (up to
+// 4,096 documents: one CTA per sequence, no cross-CTA merge). A batch
 // of 32 new keys is first tested against the 16th key with one ballot (after
 // the first batches almost every batch is skipped); otherwise the batch is
 // sorted by a 32-lane bitonic network and merged with the list by one
@@ -147,6 +148,10 @@ __global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(
   if (lane == 0) tickets[s] = 0u;  // ready for the next call
 }
 
+// IT batches of 32 keys per warp (kWarps * 32 * IT documents per CTA). With
+// one CTA per sequence the result is written directly, without the
+// candidate lists and the ticket.
+template <int IT>
 __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
     const uint32_t* __restrict__ doc_key, int64_t n_docs, int k, uint64_t* __restrict__ cand,
     unsigned* __restrict__ tickets, int32_t* __restrict__ top_ids, float* __restrict__ top_scores,
@@ -162,11 +167,10 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
   const uint32_t* keys = doc_key + (size_t)s * n_docs;
 
   // keys of this warp's slice, all loads issued before any merging
-  const int64_t w0 = (int64_t)part * kDocsPerCta + (int64_t)wid * kDocsPerWarp;
-  constexpr int kIt = kDocsPerWarp / 32;
-  uint64_t kv[kIt];
+  const int64_t w0 = (int64_t)part * (kWarps * 32 * IT) + (int64_t)wid * (32 * IT);
+  uint64_t kv[IT];
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
+  for (int it = 0; it < IT; ++it) {
     const int64_t doc = w0 + it * 32 + lane;
     kv[it] = 0;
     if (doc < n_docs) {
@@ -177,13 +181,17 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
   }
   uint64_t list = warp_sort32_desc(kv[0], lane);
 #pragma unroll
-  for (int it = 1; it < kIt; ++it) warp_fold32(list, kv[it], lane);
+  for (int it = 1; it < IT; ++it) warp_fold32(list, kv[it], lane);
   if (lane < 16) s_lists[wid][lane] = list;
   __syncthreads();
   if (wid == 0) {
     uint64_t merged = lane < 16 ? s_lists[0][lane] : 0ull;
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) merged = warp_merge16(merged, lane < 16 ? s_lists[w][lane] : 0ull, lane);
+    if (n_parts == 1) {  // the whole sequence in this CTA
+      if (lane < k) write_result(merged, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
+      return;
+    }
     if (lane < 16) cand[((size_t)s * n_parts + part) * 16 + lane] = merged;
     __threadfence();
     unsigned t = 0;
@@ -384,9 +392,23 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
     uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
     unsigned* tickets = reinterpret_cast<unsigned*>(
         reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256));
-    dim3 grid((unsigned)parts, (unsigned)n_seq);
-    cudaError_t e = launch_pdl(k <= 16 ? topk16_kernel : topk_warp_kernel, grid, dim3(kWarps * 32), 0, st,
-                               doc_key, n_docs, k, cand, tickets, top_ids, top_scores, all_scores);
+    cudaError_t e;
+    if (k <= 16 && n_docs <= 4 * kDocsPerCta) {  // one CTA per sequence
+      const dim3 grid(1u, (unsigned)n_seq);
+      if (n_docs <= kDocsPerCta)
+        e = launch_pdl(topk16_kernel<kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k, cand,
+                       tickets, top_ids, top_scores, all_scores);
+      else if (n_docs <= 2 * kDocsPerCta)
+        e = launch_pdl(topk16_kernel<2 * kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k,
+                       cand, tickets, top_ids, top_scores, all_scores);
+      else
+        e = launch_pdl(topk16_kernel<4 * kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k,
+                       cand, tickets, top_ids, top_scores, all_scores);
+    } else {
+      const dim3 grid((unsigned)parts, (unsigned)n_seq);
+      e = launch_pdl(k <= 16 ? topk16_kernel<kDocsPerWarp / 32> : topk_warp_kernel, grid, dim3(kWarps * 32), 0, st,
+                     doc_key, n_docs, k, cand, tickets, top_ids, top_scores, all_scores);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "route: top-k");
     return launch_check("route: top-k");
   }

@@ -66,6 +66,45 @@ def check_sampled(bank, qr, qso, ids, sc, alls, plans, n_random=100, seed=0):
         assert unselected.max() < sc[s].min()
 
 
+def check_prefill_attention(msa, bank, ids, w, layer, seqs):
+    """Gather + attention of a prefill call (each sequence's prefill rows are
+    its local keys, causal) in the launch configuration bench.py times, against
+    the oracle on the listed sequences."""
+    S, R = ids.shape[0], w.prefill_rows
+    q = host_normal((S * R, w.hq, 128), synth.tid("q_att", layer, 1))
+    kl = host_normal((S * R, w.hkv, 128), synth.tid("k_loc", layer, 1))
+    vl = host_normal((S * R, w.hkv, 128), synth.tid("v_loc", layer, 1))
+    cap = S * w.top_k * bank.layer_c.max_doc_chunks
+    top_d = torch.from_numpy(ids).cuda()
+    sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    sel = torch.empty(cap, dtype=torch.int64, device="cuda")
+    msa.gather(bank.layer_c, top_d, w.top_k, sel_off, sel)
+    qso = np.arange(S + 1, dtype=np.int32) * R
+    args = (from_bits(q), qso, np.zeros(S, np.int32), from_bits(kl), from_bits(vl), qso, bank.kbar, bank.vbar,
+            sel_off, sel, cap)
+    out = torch.empty((S * R, w.hq, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((S * R, w.hq, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((S * R, w.hq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(msa.attend_workspace(*args, pos_offset=float(w.top_k)), dtype=torch.uint8, device="cuda")
+    msa.attend(*args, out, ws, out_f32=of, lse=lse, pos_offset=float(w.top_k))
+    msa.sync_check()
+    of, lse = of.cpu().numpy(), lse.cpu().numpy()
+    so = sel_off.cpu().numpy()
+    sc = sel.cpu().numpy()
+    o_off, o_sel = oracle.gather(ids, bank.dco)
+    np.testing.assert_array_equal(so, o_off)
+    np.testing.assert_array_equal(sc[:so[-1]], o_sel)
+    kh, vh = bank.host_content()
+    for s_ in seqs:
+        r = slice(s_ * R, (s_ + 1) * R)
+        ss = o_sel[o_off[s_]:o_off[s_ + 1]]
+        o_out, o_lse = oracle.attend(np.ascontiguousarray(q[r]), [0, R], [0], np.ascontiguousarray(kl[r]),
+                                     np.ascontiguousarray(vl[r]), [0, R], kh, vh, [0, ss.size], ss,
+                                     pos_offset=float(w.top_k))
+        assert np.abs(of[r] - o_out).max() <= 1e-2, s_
+        np.testing.assert_allclose(lse[r], o_lse, atol=1e-3, rtol=0)
+
+
 # ------------------------------------------------------------------ tiny
 
 def test_tiny_full(msa):
@@ -86,7 +125,7 @@ def test_1m_decode_all_layers_and_prefill(msa):
     w = synth.workload("1m")
     n_exact = 0
     for layer in range(w.n_layers):
-        bank = DevBank(w.doc_tok_off, layer, content=False)
+        bank = DevBank(w.doc_tok_off, layer, content=(layer == 0))
         qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1], w.top_k, w.n_needles,
                                                    w.hr, w.d, layer)
         ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
@@ -102,6 +141,8 @@ def test_1m_decode_all_layers_and_prefill(msa):
             assert check_topk(pid, psc, o_pid, o_psc, o_pall) == 1
             np.testing.assert_allclose(pall, o_pall, atol=1e-3, rtol=0)
             assert set(pid[0].tolist()) == set(planp.docs[0])
+            # its attention (128 rows over 16 documents + 128 causal local keys), full oracle
+            check_prefill_attention(msa, bank, pid, w, layer, seqs=[0])
         del bank
     assert n_exact >= w.n_layers - 1  # rank-k gap >= 1e-2 on (almost) every layer
 
@@ -116,6 +157,8 @@ def test_10m_prefill_and_decode_sampled(msa):
                                                w.top_k, w.n_needles, w.hr, w.d, 0, call=1)
     ids, sc, alls = route_gpu(bank, qr, qso, w.top_k)
     check_sampled(bank, qr, qso, ids, sc, alls, plan, n_random=40)
+    # the prefill attention (1,024 rows x 32 heads), three sequences against the oracle
+    check_prefill_attention(msa, bank, ids, w, 0, seqs=[0, 7, 15])
     # decode: one row per sequence; sequence 0 against the full oracle
     qd, qsd, pland = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1] * w.n_seq, w.top_k,
                                                 w.n_needles, w.hr, w.d, 0)

@@ -208,6 +208,23 @@ def test_route_many_rows_each_block(msa, block):
     np.testing.assert_allclose(alls[finite], o_all[finite], atol=1e-3, rtol=0)
 
 
+@pytest.mark.parametrize("n_docs", [900, 1800, 3500, 5000])
+def test_route_topk_paths(msa, n_docs):
+    # the top-k's single-CTA variants (up to 1,024 / 2,048 / 4,096 documents) and the multi-CTA merge
+    off = _ragged_offsets(17 + n_docs, n_docs)
+    bank = DevBank(off, 8, content=False)
+    rows = (1, 3)
+    qso = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    qr = host_normal((sum(rows), 8, 128), synth.tid("q_noise", 8, n_docs))
+    ids, sc, alls = route_gpu(bank, qr, qso, 16)
+    o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, 16)
+    check_topk(ids, sc, o_ids, o_sc, o_all)
+    # the selection is the exact top-16 of the GPU's own scores (ties to the lower id)
+    for s_ in range(len(rows)):
+        order = np.lexsort((np.arange(alls.shape[1]), -alls[s_].astype(np.float64)))[:16]
+        np.testing.assert_array_equal(ids[s_], order)
+
+
 def test_route_many_rows_planted(msa, score_kernel):
     off = _ragged_offsets(15, 1200)
     bank = DevBank(off, 6, content=False)
