@@ -81,6 +81,7 @@ _sig("msa_last_error", [], ctypes.c_char_p)
 _sig("msa_version", [])
 _sig("msa_debug_set_score_kernel", [ctypes.c_int])
 _sig("msa_debug_set_pf_block", [ctypes.c_int])
+_sig("msa_debug_set_pf_pair", [ctypes.c_int])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
@@ -155,6 +156,13 @@ def set_attend_kernel(which: str) -> str:
     rows); returns the previous setting. Testing control."""
     names = ["auto", "split", "tc"]
     return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
+
+
+def set_pf_pair(on: bool) -> bool:
+    """Run the many-row scorer's 192-row blocks on CTA pairs (one M = 256 MMA
+    over two SMs) or on single CTAs; returns the previous setting. Testing
+    control."""
+    return bool(_lib.msa_debug_set_pf_pair(1 if on else 0))
 
 
 def set_pf_block(rows: int) -> int:

@@ -48,14 +48,18 @@ constexpr int kHeads = 8;
 constexpr int kEpiWarp0 = 2;
 constexpr int kSmemMax = 232448;
 
-// NB query rows per block, WQ epilogue warps per TMEM lane quadrant.
-template <int NB, int WQ>
+// NB query rows per block, WQ epilogue warps per TMEM lane quadrant. PAIR:
+// two CTAs of a cluster share one M = 256 MMA (cta_group::2); each holds its
+// 128 chunks of A and half of the NB query rows of B, and receives its 128
+// lanes x NB columns of the accumulator.
+template <int NB, int WQ, bool PAIR = false>
 struct PfCfg {
   static constexpr int kEpiWarps = 4 * WQ;
   static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kEpiThreads = 32 * kEpiWarps;
   static constexpr int kA = kM * kKB * 2;            // 16 KB
-  static constexpr int kB = NB * kKB * 2;
+  static constexpr int kBRows = PAIR ? NB / 2 : NB;  // query rows of B this CTA loads
+  static constexpr int kB = kBRows * kKB * 2;
   static constexpr int kStage = kA + kB;
   static constexpr int kTBuf = 512 / NB < 4 ? 512 / NB : 4;  // TMEM accumulators
   static constexpr int kTmemCols = 512;
@@ -69,9 +73,9 @@ struct PfCfg {
   static constexpr int kFixed = 1024 + 256 + kEpiWarps * kWarpTab;
   static constexpr int kStages = (kSmemMax - kFixed) / kStage < 8 ? (kSmemMax - kFixed) / kStage : 8;
   static constexpr int kSmem = kFixed + kStages * kStage;
-  // instruction descriptor: D fp32, A/B bf16, both K-major, N = NB, M = 128
+  // instruction descriptor: D fp32, A/B bf16, both K-major, N = NB, M = 128 (256 for a pair)
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NB >> 3) << 17) |
-                                     ((uint32_t)(kM >> 4) << 24);
+                                     ((uint32_t)((PAIR ? 2 * kM : kM) >> 4) << 24);
   static_assert(kCols % 16 == 0 && kCols * WQ == NB && kStages >= 3 && kTBuf >= 2, "tile configuration");
 };
 
@@ -89,6 +93,50 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// ---- CTA pair (cluster of 2) building blocks
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;  // clears the CTA-rank bit: the leader's copy of a shared address
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of both CTAs (not .aligned: callers may arrive from different roles).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// Both CTAs load their own tiles; the bytes count on the leader's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar & kPeerMask)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Completion of the pair's MMAs, arriving on the barrier at this offset in every CTA of `mask`.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(bar), "h"(mask)
+               : "memory");
+}
+// Arrive on the barrier at this offset in CTA `cta` of the cluster.
+__device__ __forceinline__ void mbar_arrive_cta(uint32_t bar, uint32_t cta) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+      ::"r"(bar), "r"(cta)
       : "memory");
 }
 
@@ -133,11 +181,11 @@ __device__ __forceinline__ float max_tree(const float* x) {
   return t[0];
 }
 
-template <int NB, int WQ>
-__global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
+template <int NB, int WQ, bool PAIR>
+__global__ void __launch_bounds__(PfCfg<NB, WQ, PAIR>::kThreads, 1)
     score_pf_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ PfArgs a) {
-  using C = PfCfg<NB, WQ>;
+  using C = PfCfg<NB, WQ, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -159,21 +207,35 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
     }
     for (int b = 0; b < C::kTBuf; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), C::kEpiThreads);
+      mbar_init(smem_u32(&tempty[b]), C::kEpiWarps * (PAIR ? 2 : 1));  // one arrival per epilogue warp
     }
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)C::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"((uint32_t)C::kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"((uint32_t)C::kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // both CTAs' barriers exist before either side's copies or arrivals
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // work units: tiles, or tile pairs (this CTA takes tile 2u + rank)
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+  const int ustep = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+  const int n_units = PAIR ? (a.n_tiles + 1) / 2 : a.n_tiles;
   pdl_wait();  // the prologue above overlapped the previous kernel's tail
   pdl_trigger();
 
@@ -183,19 +245,27 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x)
+      for (int u = unit0; u < n_units && ok; u += ustep) {
+        const int tile = PAIR ? 2 * u + (int)rank : u;
         for (int nb = 0; nb < a.n_nb && ok; ++nb)
           for (int kb = 0; kb < 2 * kHeads; ++kb) {
             if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) { ok = false; break; }
             const uint32_t st = smem_u32(stages + s * C::kStage);
             const uint32_t fb = smem_u32(&full[s]);
-            mbar_expect_tx(fb, C::kStage);
-            tma_load_2d(st, &tmap_a, kb * kKB, tile * kM, fb);
-            tma_load_2d(st + C::kA, &tmap_b, kb * kKB, nb * NB, fb);
+            if constexpr (PAIR) {  // the leader's barrier counts both CTAs' bytes
+              if (rank == 0) mbar_expect_tx(fb, 2 * C::kStage);
+              tma_load_2d_pair(st, &tmap_a, kb * kKB, tile * kM, fb);
+              tma_load_2d_pair(st + C::kA, &tmap_b, kb * kKB, nb * NB + (int)rank * C::kBRows, fb);
+            } else {
+              mbar_expect_tx(fb, C::kStage);
+              tma_load_2d(st, &tmap_a, kb * kKB, tile * kM, fb);
+              tma_load_2d(st + C::kA, &tmap_b, kb * kKB, nb * NB, fb);
+            }
             ++issued;
             if (++s == C::kStages) { s = 0; ph ^= 1; }
           }
-      if (!ok) {  // wait (bounded) for the copies still in flight
+      }
+      if (!ok && rank == 0) {  // wait (bounded) for the copies still in flight
         const int n = issued < C::kStages ? issued : C::kStages;
         int ss = s;
         uint32_t pp = ph;
@@ -208,12 +278,12 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // ------------------------------------------------------------- MMA (the leader of a pair)
+    if (lane == 0 && rank == 0) {
       int s = 0, b = 0;
       uint32_t ph = 0, tph = 0;  // stage ring and TMEM ring phases
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x)
+      for (int u = unit0; u < n_units && ok; u += ustep)
         for (int nb = 0; nb < a.n_nb && ok; ++nb)
           for (int h = 0; h < kHeads && ok; ++h) {
             if (!mbar_wait(smem_u32(&tempty[b]), tph ^ 1, abort_flag)) { ok = false; break; }
@@ -224,16 +294,32 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * C::kStage);
 #pragma unroll
-              for (int k = 0; k < kKB / 16; ++k)
-                tc_mma(d, sw128_desc(st + k * 32), sw128_desc(st + C::kA + k * 32), C::kIdesc, (ks | k) ? 1u : 0u);
-              tc_commit(smem_u32(&empty[s]));
+              for (int k = 0; k < kKB / 16; ++k) {
+                if constexpr (PAIR)
+                  tc_mma_pair(d, sw128_desc(st + k * 32), sw128_desc(st + C::kA + k * 32), C::kIdesc,
+                              (ks | k) ? 1u : 0u);
+                else
+                  tc_mma(d, sw128_desc(st + k * 32), sw128_desc(st + C::kA + k * 32), C::kIdesc, (ks | k) ? 1u : 0u);
+              }
+              if constexpr (PAIR)
+                tc_commit_pair(smem_u32(&empty[s]), 0x3);
+              else
+                tc_commit(smem_u32(&empty[s]));
               if (++s == C::kStages) { s = 0; ph ^= 1; }
             }
-            if (ok) tc_commit(smem_u32(&tfull[b]));
+            if (ok) {
+              if constexpr (PAIR)
+                tc_commit_pair(smem_u32(&tfull[b]), 0x3);
+              else
+                tc_commit(smem_u32(&tfull[b]));
+            }
             if (++b == C::kTBuf) { b = 0; tph ^= 1; }
           }
       // Every MMA this thread issued has completed once mma_done flips.
-      tc_commit(smem_u32(mma_done));
+      if constexpr (PAIR)
+        tc_commit_pair(smem_u32(mma_done), 0x1);
+      else
+        tc_commit(smem_u32(mma_done));
       const uint64_t t0 = globaltimer();
       while (!mbar_try(smem_u32(mma_done), 0) && globaltimer() - t0 < kWaitLimitNs) {
       }
@@ -273,7 +359,8 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
     int b = 0, blk = 0;
     uint32_t tph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x) {
+    for (int u = unit0; u < n_units && ok; u += ustep) {
+      const int tile = PAIR ? 2 * u + (int)rank : u;
       const int64_t c = (int64_t)tile * kM + row;
       const bool valid = c < a.n_chunks;
       {  // key scales and document of this lane's chunk (each lane reads only its own slots)
@@ -317,7 +404,13 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
             tmem_ld_wait();
             if (cc == C::kCols / 16 - 1) {  // this warp's part of the accumulator is in registers
               tc_fence_before();
-              mbar_arrive(smem_u32(&tempty[b]));
+              __syncwarp();
+              if (lane == 0) {  // one arrival per warp, on the leader's barrier for a pair
+                if constexpr (PAIR)
+                  mbar_arrive_cta(smem_u32(&tempty[b]), 0);
+                else
+                  mbar_arrive(smem_u32(&tempty[b]));
+              }
             }
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
@@ -401,10 +494,16 @@ __global__ void __launch_bounds__(PfCfg<NB, WQ>::kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // the leader's MMAs are done and neither CTA still reads the other's memory
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kTmemCols));
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kTmemCols));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kTmemCols));
   }
 }
 
@@ -433,11 +532,11 @@ bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NB, int WQ>
+template <int NB, int WQ, bool PAIR = false>
 msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
-  using C = PfCfg<NB, WQ>;
+  using C = PfCfg<NB, WQ, PAIR>;
   CUtensorMap ma, mb;
-  if (!make_map_2d(&ma, p.kbar_r, p.n_chunks, kM) || !make_map_2d(&mb, p.qr, p.n_rows, NB))
+  if (!make_map_2d(&ma, p.kbar_r, p.n_chunks, kM) || !make_map_2d(&mb, p.qr, p.n_rows, C::kBRows))
     return fail(MSA_ERR_CUDA, "route: cannot encode TMA tensor maps (cuTensorMapEncodeTiled)");
   PfArgs a{};
   a.invk = p.kr_inv_norm;
@@ -454,14 +553,35 @@ msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
-        cudaFuncSetAttribute(score_pf_kernel<NB, WQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaFuncSetAttribute(score_pf_kernel<NB, WQ, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return cuda_fail(e, "route: many-row scorer shared memory");
     attr_set = true;
   }
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = a.n_tiles < sms ? a.n_tiles : sms;
-  cudaError_t e = launch_pdl(score_pf_kernel<NB, WQ>, dim3(grid), dim3(C::kThreads), (size_t)C::kSmem, st, ma, mb, a);
+  cudaError_t e;
+  if constexpr (PAIR) {  // clusters of 2 CTAs, one tile pair per cluster at a time
+    const int pairs = (a.n_tiles + 1) / 2;
+    const int clusters = pairs < sms / 2 ? pairs : sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = (size_t)C::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, score_pf_kernel<NB, WQ, PAIR>, ma, mb, a);
+  } else {
+    const int grid = a.n_tiles < sms ? a.n_tiles : sms;
+    e = launch_pdl(score_pf_kernel<NB, WQ, PAIR>, dim3(grid), dim3(C::kThreads), (size_t)C::kSmem, st, ma, mb, a);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "route: score (tensor cores, many rows)");
   return launch_check("route: score (tensor cores, many rows)");
 }
@@ -475,6 +595,10 @@ bool score_pf_supported(const RoutePlan& p) {
 }
 
 int g_pf_block = 0;  // testing control: force a row block (0 = choose)
+// 192-row blocks on CTA pairs (1) or single CTAs (0, the default: measured on
+// a 161K-chunk bank with 1,024 rows the pair takes 625 us against 393 us; both
+// SMs' epilogues gate one MMA, so each step waits for the slower of the two).
+int g_pf_pair = 0;
 
 msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st) {
   // The row block with the least estimated time: padded columns times the
@@ -492,7 +616,7 @@ msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st) {
   if (g_pf_block) best = g_pf_block;
   if (best == 64) return launch_nb<64, 2>(p, st);
   if (best == 160) return launch_nb<160, 2>(p, st);
-  if (best == 192) return launch_nb<192, 3>(p, st);
+  if (best == 192) return g_pf_pair ? launch_nb<192, 3, true>(p, st) : launch_nb<192, 3>(p, st);
   return launch_nb<128, 2>(p, st);
 }
 
@@ -501,6 +625,12 @@ msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st) {
 // Forces the many-row scorer's row block (64, 128, 160 or 192; 0 = choose by
 // padding) for later route calls in this process; returns the previous
 // setting. A testing and benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_pf_pair(int on) {
+  const int old = msa::g_pf_pair;
+  if (on == 0 || on == 1) msa::g_pf_pair = on;
+  return old;
+}
+
 extern "C" int msa_debug_set_pf_block(int nb) {
   const int old = msa::g_pf_block;
   if (nb == 0 || nb == 64 || nb == 128 || nb == 160 || nb == 192) msa::g_pf_block = nb;

@@ -186,8 +186,8 @@ def test_route_many_rows_matches_oracle(msa, score_kernel, rows):
     assert np.all(np.isneginf(alls[~finite]))
 
 
-@pytest.mark.parametrize("block", [64, 128, 160, 192])
-def test_route_many_rows_each_block(msa, block):
+@pytest.mark.parametrize("block,pair", [(64, False), (128, False), (160, False), (192, False), (192, True)])
+def test_route_many_rows_each_block(msa, block, pair):
     # every row-block variant of the many-row scorer, ragged sequences across blocks
     if not msa.tc_available():
         pytest.skip("tensor-core scoring kernel not compiled in")
@@ -196,12 +196,13 @@ def test_route_many_rows_each_block(msa, block):
     rows = (100, 1, 300, 7, 200)
     qso = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
     qr = host_normal((sum(rows), 8, 128), synth.tid("q_noise", 7, 93))
-    old_k, old_b = msa.set_score_kernel("tc_rows"), msa.set_pf_block(block)
+    old_k, old_b, old_p = msa.set_score_kernel("tc_rows"), msa.set_pf_block(block), msa.set_pf_pair(pair)
     try:
         ids, sc, alls = route_gpu(bank, qr, qso, 16)
     finally:
         msa.set_score_kernel(old_k)
         msa.set_pf_block(old_b)
+        msa.set_pf_pair(old_p)
     o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, 16)
     check_topk(ids, sc, o_ids, o_sc, o_all)
     finite = np.isfinite(o_all)
@@ -223,6 +224,26 @@ def test_route_topk_paths(msa, n_docs):
     for s_ in range(len(rows)):
         order = np.lexsort((np.arange(alls.shape[1]), -alls[s_].astype(np.float64)))[:16]
         np.testing.assert_array_equal(ids[s_], order)
+
+
+@pytest.mark.parametrize("n_docs,rows", [(300, (200, 1, 90)), (1000, (192,)), (2500, (64,) * 16)])
+def test_route_cta_pair_scorer(msa, n_docs, rows):
+    # 192-row blocks on CTA pairs: odd and even tile counts, row blocks with ragged tails, planted sets
+    off = _ragged_offsets(31 + n_docs, n_docs)
+    bank = DevBank(off, 9, content=False)
+    old_k, old_b, old_p = msa.set_score_kernel("tc_rows"), msa.set_pf_block(192), msa.set_pf_pair(True)
+    try:
+        qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, list(rows), 16, 2, 8, 128, 9)
+        ids, sc, alls = route_gpu(bank, qr, qso, 16)
+    finally:
+        msa.set_score_kernel(old_k)
+        msa.set_pf_block(old_b)
+        msa.set_pf_pair(old_p)
+    o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, 16)
+    assert check_topk(ids, sc, o_ids, o_sc, o_all) == len(rows)
+    np.testing.assert_allclose(alls, o_all, atol=1e-3, rtol=0)
+    for s_ in range(len(rows)):
+        assert set(ids[s_].tolist()) == set(plan.docs[s_])
 
 
 def test_route_many_rows_planted(msa, score_kernel):
