@@ -243,8 +243,9 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   s = launch_qprep(p, eps, st);
   if (s != MSA_OK) return s;
   if (b->n_chunks > 0) {
-    // automatic: many rows -> the folded-scale contraction, a few -> per-head
-    // tensor-core accumulators, other head counts -> CUDA cores
+    // automatic: many rows -> heads in turn with the scales in the epilogue
+    // (score_pf.cu), a few -> all heads' accumulators at once (score_tc.cu),
+    // other head counts -> CUDA cores
     int which = g_score_kernel;
     if (which == 0)
       which = score_pf_supported(p) && n_rows > kManyRows ? 3 : score_tc_supported(p) ? 2 : 1;
