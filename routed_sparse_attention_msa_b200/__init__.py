@@ -82,6 +82,7 @@ _sig("msa_version", [])
 _sig("msa_debug_set_score_kernel", [ctypes.c_int])
 _sig("msa_debug_set_pf_block", [ctypes.c_int])
 _sig("msa_debug_set_pf_pair", [ctypes.c_int])
+_sig("msa_debug_wait_probe", [ctypes.c_void_p])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
@@ -156,6 +157,13 @@ def set_attend_kernel(which: str) -> str:
     rows); returns the previous setting. Testing control."""
     names = ["auto", "split", "tc"]
     return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
+
+
+def wait_probe() -> None:
+    """Launch a kernel whose bounded wait runs out (nothing arrives on its
+    barrier); the next sync_check raises with MSA_ERR_TIMEOUT. Testing control
+    for the failure path."""
+    _check(_lib.msa_debug_wait_probe(_stream(None)), "wait_probe")
 
 
 def set_pf_pair(on: bool) -> bool:

@@ -431,6 +431,12 @@ msa_status msa_attend_backward(const msa_attend_args* a, const float* dout, floa
   return launch_attend_backward(*a, dout, dq, dk_loc, dv_loc, dmem_k, dmem_v, ws, (cudaStream_t)stream);
 }
 
+// Launches a kernel whose bounded mbarrier wait runs out (nothing arrives),
+// so that the failure path can be tested without faulting the GPU: the next
+// msa_sync_check reports MSA_ERR_TIMEOUT and the context stays usable. A
+// testing control; not declared in msa.h.
+msa_status msa_debug_wait_probe(void* stream) { return launch_wait_probe((cudaStream_t)stream); }
+
 msa_status msa_sync_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaGetLastError();
