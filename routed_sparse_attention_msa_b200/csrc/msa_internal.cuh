@@ -115,7 +115,9 @@ msa_status launch_score_tc(const RoutePlan& p, cudaStream_t st);
 bool score_tc_supported(const RoutePlan& p);
 bool score_tc_built();
 int tc_error_take();  // 1 if a tensor-core kernel's bounded wait ran out since the last call
-msa_status launch_wait_probe(cudaStream_t st);  // a bounded wait that runs out (failure-path test)
+// wait_probe.cu: a bounded wait that runs out (failure-path test)
+msa_status launch_wait_probe(cudaStream_t st);
+int probe_error_take();
 // score_pf.cu: the many-row (prefill) tensor-core scorer
 msa_status launch_score_pf(const RoutePlan& p, cudaStream_t st);
 bool score_pf_supported(const RoutePlan& p);

@@ -390,27 +390,6 @@ msa_status launch_score_tc(const RoutePlan& p, cudaStream_t st) {
   return launch_nb<32>(p, st);
 }
 
-namespace {
-// A wait that nothing ends: one thread waits on an mbarrier no one arrives
-// on, the bounded wait runs out (2 s), records the error and returns.
-__global__ void wait_probe_kernel() {
-  __shared__ uint64_t bar;
-  __shared__ int abort_flag;
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bar), 1);
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0, &abort_flag);
-}
-}  // namespace
-
-msa_status launch_wait_probe(cudaStream_t st) {
-  wait_probe_kernel<<<1, 32, 0, st>>>();
-  return launch_check("wait probe");
-}
-
 int tc_error_take() {
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof v) != cudaSuccess) return 0;
