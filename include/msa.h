@@ -169,6 +169,11 @@ msa_status msa_bank_norms(const uint16_t* kbar_r, int64_t n_chunks, int32_t hr, 
  * top_ids [n_seq, k] int32 and top_scores [n_seq, k] fp32 (device).
  * all_doc_scores (device [n_seq, n_docs] fp32, or NULL) receives every score.
  * Limits: d = 128, n_seq <= 256, top_k <= 4096.
+ * How it runs (not part of the contract): with hr = 8 and up to 64 rows in a
+ * call the scorer streams the bank once with all heads' accumulators in
+ * tensor memory (bound by HBM bandwidth); above 64 rows it contracts the
+ * heads in turn on the tensor cores (bound by tensor throughput); other head
+ * counts use CUDA cores. All compute the same fp32 scores.
  * ---------------------------------------------------------------------- */
 msa_status msa_route_workspace(const msa_bank_layer* bank, int32_t n_seq, int32_t n_rows,
                                int32_t top_k, size_t* bytes);
@@ -293,6 +298,10 @@ msa_status msa_gather(const msa_gather_args* args, void* stream);
  * out is bf16 (nearest even of the fp32 result); out_f32 and lse are optional.
  * max_sel >= sel_off[s+1] - sel_off[s] for every s sizes the split-K grid.
  * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16, n_seq <= 256.
+ * How it runs (not part of the contract): when a sequence's query vectors
+ * (rows x hq / hkv) fill at least 64, the logits and P.V run on the tensor
+ * cores (the logits at fp32 accuracy, P rounded to bf16); otherwise a split-K
+ * decoding kernel on CUDA cores.
  * ---------------------------------------------------------------------- */
 typedef struct msa_attend_args {
   const uint16_t* q;          /* device [n_q, hq, d] bf16, not rotated */
