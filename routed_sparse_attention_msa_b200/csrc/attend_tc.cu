@@ -16,13 +16,13 @@
 //                 half of the block, exchanging the block max through shared
 //                 memory): running max and sum in fp32, the block's P
 //                 rounded to bf16 into shared memory,
-// When (tiles x kv heads) would not fill the GPU, the key blocks are split
-// across CTAs, each writing an unnormalised partial that the last one to
-// finish merges by log-sum-exp.
 //   O += P V      tcgen05 M128 x N128 x K64, accumulated in TMEM across
 //                 blocks (P is taken against a reference max that moves only
 //                 when the running max passes it by more than 2^11.5; then
 //                 the two threads rescale their halves of the O row in TMEM).
+// When (tiles x kv heads) would not fill the GPU, the key blocks are split
+// across CTAs, each writing an unnormalised partial that the last one to
+// finish merges by log-sum-exp.
 // The rotated queries and local keys are fp32; each is split into a bf16 high
 // part and the bf16 rounding of the remainder, and S sums Qhi Khi + Qlo Khi +
 // Qhi Klo (the Qlo Klo term is below 2^-16 of the product), so the logits keep
