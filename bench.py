@@ -45,6 +45,8 @@ def parse_args():
     p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
     p.add_argument("--score-kernel", choices=["auto", "simt", "tc", "tc_rows"], default="auto")
     p.add_argument("--attend-kernel", choices=["auto", "split", "tc"], default="auto")
+    p.add_argument("--attend-splits", type=int, default=0,
+                   help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
     p.add_argument("--content-layers", type=int, default=1,
@@ -550,6 +552,8 @@ def config_of(w, eng, args, extra=None):
                     "content": "pinned_host" if w.content_on_host else "hbm",
                     "gather": args.gather if w.content_on_host else "hbm_index",
                     "score_kernel": args.score_kernel, "attend_kernel": args.attend_kernel})
+        if args.attend_splits:
+            cfg["attend_splits"] = args.attend_splits
     else:
         cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
     cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
@@ -611,6 +615,7 @@ def run_ours(args):
     import routed_sparse_attention_msa_b200 as msa
     msa.set_score_kernel(args.score_kernel)
     msa.set_attend_kernel(args.attend_kernel)
+    msa.set_attend_splits(args.attend_splits)
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs

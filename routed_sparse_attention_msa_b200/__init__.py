@@ -84,6 +84,7 @@ _sig("msa_debug_set_pf_block", [ctypes.c_int])
 _sig("msa_debug_set_pf_pair", [ctypes.c_int])
 _sig("msa_debug_wait_probe", [ctypes.c_void_p])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
+_sig("msa_debug_set_attend_splits", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
 _sig("msa_debug_score_events", [P, P], None)
@@ -157,6 +158,13 @@ def set_attend_kernel(which: str) -> str:
     rows); returns the previous setting. Testing control."""
     names = ["auto", "split", "tc"]
     return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
+
+
+def set_attend_splits(n: int) -> int:
+    """Force the split-K attention's key splits (1..64; 0 = planned); returns
+    the previous setting. Workspace sizes follow it: query attend_workspace
+    after changing it. Benchmarking control."""
+    return int(_lib.msa_debug_set_attend_splits(int(n)))
 
 
 def wait_probe() -> None:

@@ -710,6 +710,7 @@ struct Shape {
 };
 
 int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores (testing control)
+int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
 
 // allow_tc: the forward may take the tensor-core kernel when the query
 // vectors of a sequence fill at least half of its 128-vector tile.
@@ -762,6 +763,7 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
   if (splits > cap) splits = cap;
   if (splits < 1) splits = 1;
   if (splits > 64) splits = 64;
+  if (allow_tc && g_attend_splits > 0) splits = std::min<int64_t>(g_attend_splits, std::max<int64_t>(cap, 1));
   sh.n_splits = (int)splits;
   return sh;
 }
@@ -932,5 +934,16 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
 extern "C" int msa_debug_set_attend_kernel(int which) {
   const int old = msa::g_attend_kernel;
   if (which >= 0 && which <= 2) msa::g_attend_kernel = which;
+  return old;
+}
+
+// Forces the number of key splits of the split-K forward kernel in later
+// msa_attend calls (clamped to 1..64 and to one split per 32 keys); 0 restores
+// the planned count. Returns the previous setting. Workspace sizes follow the
+// setting, so query msa_attend_workspace after changing it. A benchmarking
+// control; not declared in msa.h.
+extern "C" int msa_debug_set_attend_splits(int n) {
+  const int old = msa::g_attend_splits;
+  if (n >= 0 && n <= 64) msa::g_attend_splits = n;
   return old;
 }

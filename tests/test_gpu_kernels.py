@@ -388,6 +388,23 @@ def test_attend_staged_memory_equals_indexed(msa, attend_kernel):
     np.testing.assert_array_equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("splits", [1, 2, 5, 64])
+def test_attend_forced_splits(msa, splits):
+    """The split-K kernel with its key-split count forced (64 is clamped to one
+    split per 32 keys): splits that get no keys, one split, uneven splits."""
+    old_k, old_s = msa.set_attend_kernel("split"), msa.set_attend_splits(splits)
+    try:
+        c = _attend_case(rows=(1, 1, 2), n_loc=(65, 1, 9), n_mem=(0, 300, 61), q_start=(64, 0, 7), layer=23)
+        g_out, g_f32, g_lse = _attend_gpu(msa, c, 16.0)
+    finally:
+        msa.set_attend_splits(old_s)
+        msa.set_attend_kernel(old_k)
+    o_out, o_lse = oracle.attend(**c, pos_offset=16.0)
+    assert np.abs(g_f32 - o_out).max() <= 1e-2
+    np.testing.assert_array_equal(g_out, synth.bf16_bits(g_f32))
+    np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
+
+
 # ------------------------------------------------------- whole step, tiny
 
 def test_tiny_step_route_gather_attend(msa):
