@@ -252,6 +252,10 @@ msa_status msa_route_static(const msa_bank_layer* bank, const uint16_t* qr, cons
  *   MSA_GATHER_DEVICE_PULL: a kernel on `stream` reads the rows straight from
  *     the mapped pinned host memory; nothing waits on the host.
  * cap must be >= n_seq * min(top_k, n_docs) * bank->max_doc_chunks.
+ * Exception to the no-enqueue-on-error rule, copy-engine mode only: the ids
+ * are known only after the wait, so MSA_ERR_TIMEOUT and an out-of-range id
+ * (MSA_ERR_INVALID_ARG) leave the chunk listing and the copy of the ids
+ * enqueued on `stream`; no K-bar/V-bar copy has been issued.
  * ---------------------------------------------------------------------- */
 typedef enum msa_gather_mode {
   MSA_GATHER_COPY_ENGINE = 0,

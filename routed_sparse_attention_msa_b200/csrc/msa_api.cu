@@ -287,10 +287,17 @@ msa_status msa_gather(const msa_gather_args* a, void* stream) {
   if (a->cap < need)
     return fail(MSA_ERR_CAPACITY, "gather: cap = %lld < n_seq * k * max_doc_chunks = %lld", (long long)a->cap,
                 (long long)need);
+  if (b.content_on_host) {  // checked before anything is enqueued
+    if (!a->stage_k || !a->stage_v) return fail(MSA_ERR_INVALID_ARG, "gather: staging buffers required for host content");
+    if (a->mode != MSA_GATHER_DEVICE_PULL && a->mode != MSA_GATHER_COPY_ENGINE)
+      return fail(MSA_ERR_INVALID_ARG, "gather: unknown mode %d", a->mode);
+    if (a->mode == MSA_GATHER_COPY_ENGINE &&
+        (!a->doc_chunk_off_host || !a->top_ids_host || !a->copy_stream || !a->done_event))
+      return fail(MSA_ERR_INVALID_ARG, "gather: copy-engine mode needs doc_chunk_off_host, top_ids_host, copy_stream, done_event");
+  }
   cudaStream_t st = (cudaStream_t)stream;
   s = launch_gather_index(b, a->top_ids, a->n_seq, k, a->sel_off, a->sel_chunk, st);
   if (s != MSA_OK || !b.content_on_host) return s;
-  if (!a->stage_k || !a->stage_v) return fail(MSA_ERR_INVALID_ARG, "gather: staging buffers required for host content");
   if (a->mode == MSA_GATHER_DEVICE_PULL) {
     // The kernel reads the pinned host rows through their device-side mapping.
     msa_bank_layer mapped = b;
@@ -303,9 +310,6 @@ msa_status msa_gather(const msa_gather_args* a, void* stream) {
     mapped.vbar = static_cast<const uint16_t*>(dv);
     return launch_gather_pull(mapped, a->sel_off + a->n_seq, a->sel_chunk, a->cap, a->stage_k, a->stage_v, st);
   }
-  if (a->mode != MSA_GATHER_COPY_ENGINE) return fail(MSA_ERR_INVALID_ARG, "gather: unknown mode %d", a->mode);
-  if (!a->doc_chunk_off_host || !a->top_ids_host || !a->copy_stream || !a->done_event)
-    return fail(MSA_ERR_INVALID_ARG, "gather: copy-engine mode needs doc_chunk_off_host, top_ids_host, copy_stream, done_event");
   const size_t ids_bytes = (size_t)a->n_seq * k * sizeof(int32_t);
   cudaError_t e = cudaMemcpyAsync(a->top_ids_host, a->top_ids, ids_bytes, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather: copy ids to host");
@@ -319,12 +323,14 @@ msa_status msa_gather(const msa_gather_args* a, void* stream) {
     if (timed_out(t0, limit)) return fail(MSA_ERR_TIMEOUT, "gather: ids not ready after %lld us", (long long)limit);
     std::this_thread::yield();
   }
+  for (int i = 0; i < a->n_seq * k; ++i)  // every id checked before the first copy is issued
+    if (a->top_ids_host[i] < 0 || a->top_ids_host[i] >= b.n_docs)
+      return fail(MSA_ERR_INVALID_ARG, "gather: document id %d out of range", a->top_ids_host[i]);
   cudaStream_t cs = (cudaStream_t)a->copy_stream;
   const size_t row = (size_t)b.hkv * kHeadDim;
   int64_t dst = 0;
   for (int i = 0; i < a->n_seq * k; ++i) {
     const int32_t doc = a->top_ids_host[i];
-    if (doc < 0 || doc >= b.n_docs) return fail(MSA_ERR_INVALID_ARG, "gather: document id %d out of range", doc);
     int64_t c0 = a->doc_chunk_off_host[doc], c1 = a->doc_chunk_off_host[doc + 1];
     // merge with following ranks whose chunks continue this range
     while (i + 1 < a->n_seq * k && c1 == a->doc_chunk_off_host[a->top_ids_host[i + 1]] &&
