@@ -44,6 +44,10 @@
  *    a message for the calling thread's last failure. Errors raised by kernels
  *    after launch surface at the next CUDA synchronisation (msa_sync_check).
  *  - No C++ exception crosses this interface.
+ *  - One GPU per process: the kernels' shared-memory limits are raised on the
+ *    device current at their first launch in the process, so calls on a
+ *    second device of the same process can fail with MSA_ERR_CUDA. Run one
+ *    process per GPU (msa_route_static's scratch lookup is per device).
  */
 #ifndef MSA_H
 #define MSA_H
