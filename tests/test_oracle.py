@@ -282,6 +282,19 @@ def test_route_scores_are_cosines_in_range_and_scale_invariant():
     np.testing.assert_allclose(ds2, ds, atol=1e-14)
 
 
+def test_route_each_norm_is_clamped_at_eps():
+    # With eps = 0.5 a vector shorter than eps counts as if it had length eps:
+    # for parallel q and k the score is |q| |k| / (max(|q|, eps) max(|k|, eps)),
+    # exactly 1 when both are longer than eps and proportionally less when not.
+    hr, d = 4, 32
+    e = np.zeros((hr, d))
+    e[np.arange(hr), 3 * np.arange(hr)] = 1.0  # one unit direction per head
+    kbar = np.stack([2.0 * e, 0.25 * e, np.roll(e, 1, axis=1)])  # docs: long, short, orthogonal
+    qr = np.stack([0.25 * e, 2.0 * e])  # sequence 0: a short row, sequence 1: a long row
+    _, _, ds = oracle.route(bf(kbar), [0, 1, 2, 3], bf(qr), [0, 1, 2], top_k=3, eps=0.5)
+    np.testing.assert_allclose(ds, [[0.5, 0.25, 0.0], [1.0, 0.5, 0.0]], atol=1e-15)
+
+
 def test_route_mean_over_heads():
     # Two heads; the second query head is the zero vector, so it contributes
     # nothing and every score is half the first head's cosine.

@@ -50,6 +50,35 @@ MUTANTS = {
     "bf16_truncate": ("double r = nearbyint(ldexp(ax, -q));", "double r = floor(ldexp(ax, -q));"),
     "gather_skips_last_chunk": ("for (int64_t c = doc_chunk_off[doc]; c < doc_chunk_off[doc + 1]; ++c) {",
                                 "for (int64_t c = doc_chunk_off[doc]; c + 1 < doc_chunk_off[doc + 1]; ++c) {"),
+    "gather_reverse_rank": ("int32_t doc = top_ids[(size_t)s * top_k + i];",
+                            "int32_t doc = top_ids[(size_t)s * top_k + (top_k - 1 - i)];"),
+    "encode_rotates_v": ("for (int i = 0; i < d; ++i) sv[(size_t)h * d + i] += orc_bf16_to_double(vs[i]);",
+                         "{ double w[1024]; for (int i = 0; i < d; ++i) w[i] = orc_bf16_to_double(vs[i]); "
+                         "orc_rope(w, d, (double)p, rope_theta); for (int i = 0; i < d; ++i) sv[(size_t)h * d + i] += w[i]; }"),
+    "encode_rotates_kr": ("for (int i = 0; i < d; ++i) sr[(size_t)h * d + i] += orc_bf16_to_double(rs[i]);",
+                          "{ double w[1024]; for (int i = 0; i < d; ++i) w[i] = orc_bf16_to_double(rs[i]); "
+                          "orc_rope(w, d, (double)p, rope_theta); for (int i = 0; i < d; ++i) sr[(size_t)h * d + i] += w[i]; }"),
+    "encode_v_full_chunk_divisor": ("vbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sv[i] / (double)n);",
+                                    "vbar[(size_t)c * hkv * d + i] = orc_double_to_bf16(sv[i] / (double)chunk);"),
+    "route_missing_qnorm": ("cos_sum += dot * inv_q[h] * inv_k[h];", "cos_sum += dot * inv_k[h];"),
+    "route_norm_eps_added": ("inv[(size_t)r * hr + h] = 1.0 / (nrm > eps ? nrm : eps);",
+                             "inv[(size_t)r * hr + h] = 1.0 / (nrm + eps);"),
+    "route_first_row_only": ("for (int64_t t = q_seq_off[s]; t < q_seq_off[s + 1]; ++t) {",
+                             "for (int64_t t = q_seq_off[s]; t < q_seq_off[s] + 1; ++t) {"),
+    "attend_memory_keys_rotated": ("gidx[n++] = sel_off[s] + m;",
+                                   "{ orc_rope(keys + (size_t)n * d, d, pos_offset, rope_theta); double t2 = 0.0; "
+                                   "for (int i = 0; i < d; ++i) t2 += qv[i] * keys[(size_t)n * d + i]; "
+                                   "logit[n] = t2 * scale; } gidx[n++] = sel_off[s] + m;"),
+    "attend_local_keys_no_offset": ("orc_rope(kv, d, pos_offset + (double)j, rope_theta);",
+                                    "orc_rope(kv, d, (double)j, rope_theta);"),
+    "attend_values_from_keys": ("for (int i = 0; i < d; ++i) o[i] += p * orc_ld(vv, voff[j] + i);",
+                                "for (int i = 0; i < d; ++i) o[i] += p * orc_ld(vsrc[j] ? k_loc : mem_k, voff[j] + i);"),
+    "attend_q_start_ignored": ("int64_t gq = (int64_t)q_start[s] + (r - q_seq_off[s]);",
+                               "int64_t gq = (int64_t)(r - q_seq_off[s]);"),
+    "bf16_ties_away": ("double r = nearbyint(ldexp(ax, -q));", "double r = round(ldexp(ax, -q));"),
+    "backward_memory_key_rotated_back": ("for (int i = 0; i < d; ++i) dk[i] += scale * ds * qv[i];\n          }",
+                                         "double w[1024]; for (int i = 0; i < d; ++i) w[i] = scale * ds * qv[i]; "
+                                         "orc_rope(w, d, -pos_offset, rope_theta); for (int i = 0; i < d; ++i) dk[i] += w[i];\n          }"),
 }
 
 PIN_TESTS = ([getattr(pins, n) for n in dir(pins) if n.startswith("test_")] +
