@@ -12,13 +12,13 @@
  *               every pooled routing key, mean over heads, max over the
  *               sequence's rows and the document's chunks, top-k documents.
  *               ["MSA: Memory Sparse Attention", Overall Design: Architecture
- *               ("mean-pooled over heads, then token-wise max", Top-k);
+ *               (head mean first, then the max over query tokens; Top-k);
  *               "MSA-arXiv26", 核心方法 (cosine similarity, top-k documents)]
  *   msa_gather  context assembly: the chunk list of the selected documents,
  *               and their pooled K/V fetched from pinned host memory when the
  *               content tier lives there.
  *               ["MSA: Memory Sparse Attention", Inference Pipeline stage 2
- *               ("load only the selected K/V") and the Memory Parallel
+ *               (only the selected documents' pooled K/V are loaded) and the Memory Parallel
  *               paragraph (content K/V in host DRAM, fetched asynchronously);
  *               "MSA-arXiv26", 核心方法 / Memory Parallel inference (tiered storage)]
  *   msa_attend  sparse attention of every query row over the selected pooled
@@ -190,9 +190,9 @@ msa_status msa_route(const msa_bank_layer* bank, const uint16_t* qr, const int32
 /* ------------------------------------------------------------------------
  * Merge of per-shard top-k lists (Memory Parallel).
  *
- * ["MSA: Memory Sparse Attention", Inference Pipeline: Memory Parallel shards
- * the routing keys across GPUs — query broadcast, local scoring, global
- * reduce; "MSA-arXiv26", 核心方法 / Memory Parallel inference]
+ * ["MSA: Memory Sparse Attention", Inference Pipeline: Memory Parallel splits
+ * the routing keys over GPUs, each scores the query against its part and the
+ * results are combined; "MSA-arXiv26", 核心方法 / Memory Parallel inference]
  *
  * When the documents are split into n_shards contiguous ranges, each routed
  * by msa_route on its own bank (local document ids), shard g's lists

@@ -8,8 +8,8 @@ single-threaded, fp64 sums, loops in the order of the definitions.
 Definitions followed (page title, section):
   * "MSA: Memory Sparse Attention" (project README), Overall Design,
     Architecture and Figure 2: chunk-mean pooled K/V/K_r, cosine routing
-    (mean over heads, then token-wise max), top-k documents, concatenation of
-    their compressed K/V with the query's local K/V; parallel (document-wise)
+    (head mean, then the max over query tokens), top-k documents, the selected
+    pooled K/V joined to the query's own recent K/V; parallel (document-wise)
     RoPE from 0 and global RoPE offset by k.
   * same page, Inference Pipeline and Figure 3: offline encoding of
     (K-bar, V-bar, K-bar_r), online routing, loading only the selected K/V.

@@ -215,8 +215,8 @@ static double orc_chunk_score(orc_arr kr, int64_t c, orc_arr q, int64_t t, int h
   return cos_sum / (double)hr; /* mean over heads */
 }
 
-/* [P2] Architecture: relevance by cosine similarity, mean-pooled over heads,
- * then token-wise max; the top-k documents are selected. [P1] 核心方法: the
+/* [P2] Architecture: relevance is a cosine similarity averaged over the heads
+ * and then maximised over query tokens; the top-k documents are selected. [P1] 核心方法: the
  * query is compared with every document's pooled routing keys.
  * Readings: the max runs over the sequence's query rows and the document's
  * chunks; each norm is clamped separately at eps; ties go to the lower id. */
@@ -361,8 +361,8 @@ int64_t orc_gather(const int32_t* top_ids, int n_seq, int top_k, const int64_t* 
 
 /* ------------------------------------------------------------------ attend */
 
-/* [P2] Architecture: the selected documents' compressed K/V are concatenated
- * with the query's local K/V; global RoPE offsets the query's start index by k,
+/* [P2] Architecture: the selected documents' pooled K/V are joined to the
+ * K/V of the query's own recent context; global RoPE shifts the query by k,
  * keeping the order background -> query -> generation. Readings: every query
  * row sees every selected pooled key; local keys are causal (row g sees local
  * j <= g); q head h uses kv head h / (hq / hkv); logits are scaled by `scale`.

@@ -3,8 +3,8 @@
 // concatenated with its local K/V, with the query and the local keys rotated
 // at global positions offset by k; GQA; causal over the local keys.
 //
-// ["MSA: Memory Sparse Attention", Overall Design: Architecture — the selected
-// documents' compressed K/V are concatenated with the query's local K/V;
+// ["MSA: Memory Sparse Attention", Overall Design: Architecture — the pooled
+// K/V of the selected documents joined to the K/V of the query's recent context;
 // Parallel (document-wise) RoPE and Global RoPE offset by k (Figure 2)]
 //
 // Two kernels:

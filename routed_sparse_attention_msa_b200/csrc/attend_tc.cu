@@ -1,8 +1,8 @@
 // Sparse attention for many query rows per sequence (prefill), on the tensor
 // cores.
 //
-// ["MSA: Memory Sparse Attention", Overall Design: Architecture — the selected
-// documents' compressed K/V are concatenated with the query's local K/V;
+// ["MSA: Memory Sparse Attention", Overall Design: Architecture — the pooled
+// K/V of the selected documents joined to the K/V of the query's recent context;
 // Parallel (document-wise) RoPE and Global RoPE offset by k (Figure 2)]
 //
 // Same result as the split-K kernel in attend.cu (which stays the decoding

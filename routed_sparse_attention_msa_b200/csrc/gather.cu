@@ -2,10 +2,10 @@
 // and (host content tier, device-pull mode) the copy of their pooled K/V rows
 // from mapped pinned host memory into a device staging buffer.
 //
-// ["MSA: Memory Sparse Attention", Inference Pipeline stage 2 — load only the
-// selected K-bar/V-bar and concatenate with local context; the Memory Parallel
-// paragraph — content K-bar/V-bar stays in host DRAM and is fetched when
-// selected; "MSA-arXiv26", 核心方法 / Memory Parallel inference (tiered storage)]
+// ["MSA: Memory Sparse Attention", Inference Pipeline stage 2 — only the
+// selected documents' K-bar/V-bar are brought in and joined to the local
+// context; the Memory Parallel paragraph — the content tier is kept in host
+// memory and read on selection; "MSA-arXiv26", 核心方法 / Memory Parallel inference (tiered storage)]
 #include "msa_internal.cuh"
 
 namespace msa {

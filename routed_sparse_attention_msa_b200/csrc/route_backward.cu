@@ -1,9 +1,8 @@
 // Gradient of the routing scores, for the contrastive routing loss that
 // trains the routing projectors end to end.
 //
-// ["MSA: Memory Sparse Attention", Abstract and Key Contributions — an
-// end-to-end trainable sparse attention, top-k selection fused with sparse
-// attention; "MSA-arXiv26", 核心方法 — generation loss plus a contrastive
+// ["MSA: Memory Sparse Attention", Abstract and Key Contributions — sparse
+// attention whose document selection is trained jointly with the model; "MSA-arXiv26", 核心方法 — generation loss plus a contrastive
 // routing loss]
 //
 // score(s, j) = max over rows t of s and chunks c of j of

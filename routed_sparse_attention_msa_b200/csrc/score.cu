@@ -2,7 +2,7 @@
 // scoring kernels.
 //
 // ["MSA: Memory Sparse Attention", Overall Design: Architecture — relevance by
-// cosine similarity, mean over heads, then token-wise max; "MSA-arXiv26",
+// cosine similarity, averaged over heads, then maximised over query tokens; "MSA-arXiv26",
 // 核心方法 — the query is compared with every document's pooled routing key]
 //
 // score(s, j) = max over rows t of s, chunks c of j, of

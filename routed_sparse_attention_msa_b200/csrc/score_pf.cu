@@ -1,7 +1,7 @@
 // Routing scores of many query rows at once (prefill), on the tensor cores.
 //
 // ["MSA: Memory Sparse Attention", Overall Design: Architecture — cosine
-// similarity mean-pooled over heads, then token-wise max; "MSA-arXiv26",
+// similarity averaged over heads, then maximised over query tokens; "MSA-arXiv26",
 // 核心方法 — the query scored against every document's pooled routing keys]
 //
 //   score(s, j) = max over rows t of s and chunks c of j of

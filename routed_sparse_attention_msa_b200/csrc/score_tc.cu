@@ -1,7 +1,7 @@
 // Routing scores on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
 //
 // ["MSA: Memory Sparse Attention", Overall Design: Architecture — relevance by
-// cosine similarity, mean-pooled over heads, then token-wise max; Top-k
+// cosine similarity, averaged over heads, then maximised over query tokens; Top-k
 // documents. "MSA-arXiv26", 核心方法 — the query is scored against every
 // document's pooled routing keys]
 //

@@ -4,8 +4,9 @@ ids), the k candidates of every sequence are all-gathered, and every rank
 merges them with ``topk_merge`` into the global top-k, identical to routing
 the unsharded bank.
 
-["MSA: Memory Sparse Attention", Inference Pipeline: Memory Parallel shards
-the routing keys across GPUs (query broadcast, local scoring, global reduce);
+["MSA: Memory Sparse Attention", Inference Pipeline: Memory Parallel splits
+the routing keys over GPUs, each scores the query against its part, and the
+results are reduced;
 "MSA-arXiv26", 核心方法 / Memory Parallel inference]
 
 Host-side planning and collective plumbing only; the scoring and the merge
