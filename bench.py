@@ -68,6 +68,9 @@ def parse_args():
                    help="replay each step as one CUDA graph (auto: on unless the copy-engine gather needs host syncs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--stage-times", action="store_true",
+                   help="after the timed region, time route / gather / attend separately (CUDA events around "
+                        "each call, eager launches, warm) and report them per layer in config")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="only run warmup + this many steps, no extra legs (for ncu captures)")
     return p.parse_args()
@@ -187,6 +190,38 @@ def combine_ranks(ms: float, units_per_step: float, world: int, device="cuda"):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     return units_per_step * world / (ms / 1e3), ms
+
+
+class StageClock:
+    """Stands in for the binding during a diagnostic pass: records CUDA events
+    on the caller's current stream around each route, gather and attend call
+    (the stream the library enqueues on) and keeps them for summing later."""
+
+    STAGES = ("route", "gather", "attend")
+
+    def __init__(self, msa, torch):
+        self._msa, self._torch = msa, torch
+        self.marks = []  # (stage, start event, end event)
+
+    def __getattr__(self, name):
+        f = getattr(self._msa, name)
+        if name not in self.STAGES:
+            return f
+
+        def timed(*a, **k):
+            s = self._torch.cuda.Event(enable_timing=True)
+            e = self._torch.cuda.Event(enable_timing=True)
+            s.record()
+            f(*a, **k)
+            e.record()
+            self.marks.append((name, s, e))
+        return timed
+
+    def per_call_us(self, calls: int) -> dict:
+        tot = {}
+        for name, s, e in self.marks:
+            tot[name] = tot.get(name, 0.0) + 1e3 * s.elapsed_time(e)
+        return {k: v / calls for k, v in tot.items()}
 
 
 # --------------------------------------------------------- workload engine
@@ -416,6 +451,19 @@ class Routed:
     def step(self, evs=None):
         for l in range(self.L):
             self.layer(l, None if evs is None else evs[l])
+
+    def stage_times(self, reps: int = 3) -> dict:
+        """Warm device time of each stage per layer (eager launches, events
+        around every call), for a breakdown of the step."""
+        clock = StageClock(self.msa, self.torch)
+        real, self.msa = self.msa, clock
+        try:
+            for _ in range(reps):
+                self.step()
+        finally:
+            self.msa = real
+        self.torch.cuda.synchronize()
+        return clock.per_call_us(reps * self.L)
 
     def units_per_step(self) -> float:
         return float(self.w.memory_tokens) * self.S * self.L
@@ -749,6 +797,8 @@ def run_ours(args):
                               f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
 
     extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None, "mode": args.mode}
+    if args.stage_times and w.name != "encode":
+        extra["stage_us_per_layer"] = eng.stage_times()
     if args.mode == "sharded":
         extra["shards"] = args.shards
     if args.mode == "interleave":
