@@ -786,14 +786,10 @@ Layout layout(const msa_attend_args& a, const Shape& sh) {
 
 template <int VEC>
 msa_status launch_vec(const AttnParams& P, dim3 grid, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_split_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(Smem<VEC>));
-    if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
-    attr = true;
-  }
-  cudaError_t e = launch_pdl(attend_split_kernel<VEC>, grid, dim3(kThreads), sizeof(Smem<VEC>), st, P);
+  static std::atomic<uint64_t> attr{0};
+  cudaError_t e = smem_limit_once(attend_split_kernel<VEC>, (int)sizeof(Smem<VEC>), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
+  e = launch_pdl(attend_split_kernel<VEC>, grid, dim3(kThreads), sizeof(Smem<VEC>), st, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: split-K with merge");
   return launch_check("attend: split-K with merge");
 }
@@ -848,14 +844,10 @@ msa_status launch_rope(const AttnParams& P, const msa_attend_args& a, const Shap
 template <int VEC>
 msa_status launch_bwd_dq(const AttnParams& P, const float* dout, const float* Dvec, float* dq, dim3 grid,
                          cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_bwd_dq_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(BwdQSmem<VEC>));
-    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
-    attr = true;
-  }
-  cudaError_t e = launch_pdl(attend_bwd_dq_kernel<VEC>, grid, dim3(kThreads), sizeof(BwdQSmem<VEC>), st, P, dout,
+  static std::atomic<uint64_t> attr{0};
+  cudaError_t e = smem_limit_once(attend_bwd_dq_kernel<VEC>, (int)sizeof(BwdQSmem<VEC>), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
+  e = launch_pdl(attend_bwd_dq_kernel<VEC>, grid, dim3(kThreads), sizeof(BwdQSmem<VEC>), st, P, dout,
                              Dvec, dq);
   if (e != cudaSuccess) return cuda_fail(e, "attend backward: dq");
   return launch_check("attend backward: dq");
@@ -911,13 +903,9 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
   int max_loc = 0;
   for (int q = 0; q < a.n_seq; ++q) max_loc = std::max(max_loc, a.loc_off[q + 1] - a.loc_off[q]);
   const int64_t max_keys = a.max_sel + max_loc;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(attend_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(BwdKVSmem));
-    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  e = smem_limit_once(attend_bwd_dkdv_kernel, (int)sizeof(BwdKVSmem), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
   dim3 gk((unsigned)((max_keys + kBwdKeys - 1) / kBwdKeys > 0 ? (max_keys + kBwdKeys - 1) / kBwdKeys : 1),
           (unsigned)a.hkv, (unsigned)a.n_seq);
   e = launch_pdl(attend_bwd_dkdv_kernel, gk, dim3(kThreads), sizeof(BwdKVSmem), st, P, dout, Dvec, dk_loc, dv_loc,
