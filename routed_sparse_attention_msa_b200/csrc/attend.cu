@@ -709,7 +709,7 @@ struct Shape {
   bool tc;  // tensor-core kernel (many rows per sequence)
 };
 
-int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores (testing control)
+int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores (testing control)
 int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
 
 // allow_tc: the forward may take the tensor-core kernel when the query
@@ -722,7 +722,7 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
     const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
     max_rows = rows > max_rows ? rows : max_rows;
   }
-  sh.tc = allow_tc && g_attend_kernel != 1 && kAttnTcVec % group == 0 &&
+  sh.tc = allow_tc && g_attend_kernel != 1 && g_attend_kernel != 3 && kAttnTcVec % group == 0 &&
           (g_attend_kernel == 2 || max_rows * group >= kAttnTcVec / 2);
   if (sh.tc) {
     sh.vec = kAttnTcVec;
@@ -863,6 +863,7 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   msa_status s = launch_rope(P, a, sh, st);
   if (s != MSA_OK) return s;
   if (sh.tc) return launch_attend_tc(P, st);
+  if (g_attend_kernel == 3) return launch_attend_dec_tc(P, st);
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
     case 4: return launch_vec<4>(P, grid, st);
@@ -917,11 +918,12 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
 }  // namespace msa
 
 // Selects the attention kernel of later msa_attend calls in this process:
-// 0 = automatic, 1 = split-K, 2 = tensor cores (any row count); returns the
-// previous setting. A testing and benchmarking control; not declared in msa.h.
+// 0 = automatic, 1 = split-K, 2 = tensor cores (any row count), 3 = the
+// decoding tensor-core kernel (in place of split-K); returns the previous
+// setting. A testing and benchmarking control; not declared in msa.h.
 extern "C" int msa_debug_set_attend_kernel(int which) {
   const int old = msa::g_attend_kernel;
-  if (which >= 0 && which <= 2) msa::g_attend_kernel = which;
+  if (which >= 0 && which <= 3) msa::g_attend_kernel = which;
   return old;
 }
 

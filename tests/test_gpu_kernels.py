@@ -366,7 +366,7 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc"])
+@pytest.fixture(params=["split", "tc", "tc_dec"])
 def attend_kernel(request, msa):
     old = msa.set_attend_kernel(request.param)
     yield request.param
