@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
     p.add_argument("--score-kernel", choices=["auto", "simt", "tc", "tc_rows"], default="auto")
-    p.add_argument("--attend-kernel", choices=["auto", "split", "tc"], default="auto")
+    p.add_argument("--attend-kernel", choices=["auto", "split", "tc", "tc_dec"], default="auto")
     p.add_argument("--attend-splits", type=int, default=0,
                    help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",

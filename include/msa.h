@@ -44,10 +44,10 @@
  *    a message for the calling thread's last failure. Errors raised by kernels
  *    after launch surface at the next CUDA synchronisation (msa_sync_check).
  *  - No C++ exception crosses this interface.
- *  - One GPU per process: the kernels' shared-memory limits are raised on the
- *    device current at their first launch in the process, so calls on a
- *    second device of the same process can fail with MSA_ERR_CUDA. Run one
- *    process per GPU (msa_route_static's scratch lookup is per device).
+ *  - Several GPUs in one process are supported: every call works on the
+ *    device current on the calling thread, and per-device kernel settings
+ *    (shared-memory limits, msa_route_static's scratch address) are set up
+ *    once per device on first use.
  */
 #ifndef MSA_H
 #define MSA_H
@@ -222,7 +222,8 @@ msa_status msa_topk_merge(const int32_t* ids, const float* scores, const int64_t
  * GPU that loads the library holds until the process exits.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current). Make that first call before any
- *    stream capture.
+ *    stream capture. The address is kept for the life of the process, so
+ *    cudaDeviceReset between calls is not supported.
  *  - A call whose scratch need (msa_route_workspace) exceeds the array
  *    returns MSA_ERR_CAPACITY and enqueues nothing.
  *  - All calls on a device share the one array; it keeps the last call's

@@ -154,9 +154,10 @@ def score_events(begin, end) -> None:
 
 
 def set_attend_kernel(which: str) -> str:
-    """'auto', 'split' (split-K decoding kernel) or 'tc' (tensor cores, many
-    rows); returns the previous setting. Testing control."""
-    names = ["auto", "split", "tc"]
+    """'auto', 'split' (split-K decoding kernel), 'tc' (tensor cores, many
+    rows) or 'tc_dec' (tensor cores with the keys as M, for decoding shapes);
+    returns the previous setting. Testing control."""
+    names = ["auto", "split", "tc", "tc_dec"]
     return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
 
 

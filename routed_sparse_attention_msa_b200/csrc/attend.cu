@@ -709,7 +709,7 @@ struct Shape {
   bool tc;  // tensor-core kernel (many rows per sequence)
 };
 
-int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores (testing control)
+int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores (testing control)
 int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
 
 // allow_tc: the forward may take the tensor-core kernel when the query
@@ -722,7 +722,7 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
     const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
     max_rows = rows > max_rows ? rows : max_rows;
   }
-  sh.tc = allow_tc && g_attend_kernel != 1 && kAttnTcVec % group == 0 &&
+  sh.tc = allow_tc && g_attend_kernel != 1 && g_attend_kernel != 3 && kAttnTcVec % group == 0 &&
           (g_attend_kernel == 2 || max_rows * group >= kAttnTcVec / 2);
   if (sh.tc) {
     sh.vec = kAttnTcVec;
@@ -786,14 +786,10 @@ Layout layout(const msa_attend_args& a, const Shape& sh) {
 
 template <int VEC>
 msa_status launch_vec(const AttnParams& P, dim3 grid, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_split_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(Smem<VEC>));
-    if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
-    attr = true;
-  }
-  cudaError_t e = launch_pdl(attend_split_kernel<VEC>, grid, dim3(kThreads), sizeof(Smem<VEC>), st, P);
+  static std::atomic<uint64_t> attr{0};
+  cudaError_t e = smem_limit_once(attend_split_kernel<VEC>, (int)sizeof(Smem<VEC>), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: shared memory");
+  e = launch_pdl(attend_split_kernel<VEC>, grid, dim3(kThreads), sizeof(Smem<VEC>), st, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: split-K with merge");
   return launch_check("attend: split-K with merge");
 }
@@ -848,14 +844,10 @@ msa_status launch_rope(const AttnParams& P, const msa_attend_args& a, const Shap
 template <int VEC>
 msa_status launch_bwd_dq(const AttnParams& P, const float* dout, const float* Dvec, float* dq, dim3 grid,
                          cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_bwd_dq_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(BwdQSmem<VEC>));
-    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
-    attr = true;
-  }
-  cudaError_t e = launch_pdl(attend_bwd_dq_kernel<VEC>, grid, dim3(kThreads), sizeof(BwdQSmem<VEC>), st, P, dout,
+  static std::atomic<uint64_t> attr{0};
+  cudaError_t e = smem_limit_once(attend_bwd_dq_kernel<VEC>, (int)sizeof(BwdQSmem<VEC>), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
+  e = launch_pdl(attend_bwd_dq_kernel<VEC>, grid, dim3(kThreads), sizeof(BwdQSmem<VEC>), st, P, dout,
                              Dvec, dq);
   if (e != cudaSuccess) return cuda_fail(e, "attend backward: dq");
   return launch_check("attend backward: dq");
@@ -871,6 +863,7 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   msa_status s = launch_rope(P, a, sh, st);
   if (s != MSA_OK) return s;
   if (sh.tc) return launch_attend_tc(P, st);
+  if (g_attend_kernel == 3) return launch_attend_dec_tc(P, st);
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
     case 4: return launch_vec<4>(P, grid, st);
@@ -911,13 +904,9 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
   int max_loc = 0;
   for (int q = 0; q < a.n_seq; ++q) max_loc = std::max(max_loc, a.loc_off[q + 1] - a.loc_off[q]);
   const int64_t max_keys = a.max_sel + max_loc;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(attend_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(BwdKVSmem));
-    if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  e = smem_limit_once(attend_bwd_dkdv_kernel, (int)sizeof(BwdKVSmem), attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend backward: shared memory");
   dim3 gk((unsigned)((max_keys + kBwdKeys - 1) / kBwdKeys > 0 ? (max_keys + kBwdKeys - 1) / kBwdKeys : 1),
           (unsigned)a.hkv, (unsigned)a.n_seq);
   e = launch_pdl(attend_bwd_dkdv_kernel, gk, dim3(kThreads), sizeof(BwdKVSmem), st, P, dout, Dvec, dk_loc, dv_loc,
@@ -929,11 +918,12 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
 }  // namespace msa
 
 // Selects the attention kernel of later msa_attend calls in this process:
-// 0 = automatic, 1 = split-K, 2 = tensor cores (any row count); returns the
-// previous setting. A testing and benchmarking control; not declared in msa.h.
+// 0 = automatic, 1 = split-K, 2 = tensor cores (any row count), 3 = the
+// decoding tensor-core kernel (in place of split-K); returns the previous
+// setting. A testing and benchmarking control; not declared in msa.h.
 extern "C" int msa_debug_set_attend_kernel(int which) {
   const int old = msa::g_attend_kernel;
-  if (which >= 0 && which <= 2) msa::g_attend_kernel = which;
+  if (which >= 0 && which <= 3) msa::g_attend_kernel = which;
   return old;
 }
 

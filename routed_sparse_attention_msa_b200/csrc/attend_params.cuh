@@ -48,4 +48,10 @@ constexpr int kAttnTcVec = 128;
 msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st);
 int attend_tc_error_take();  // 1 if its bounded wait ran out since the last call
 
+// attend_dec_tc.cu: the decoding shapes (at most 16 query vectors per CTA) on
+// the tensor cores, keys as the MMA's M side; same grid and split-K plan as
+// the split-K kernel. Needs rope_rows to have run.
+msa_status launch_attend_dec_tc(const AttnParams& P, cudaStream_t st);
+int attend_dec_tc_error_take();
+
 }  // namespace msa

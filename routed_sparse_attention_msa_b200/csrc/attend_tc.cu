@@ -459,13 +459,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
 }  // namespace
 
 msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
-    if (e != cudaSuccess) return cuda_fail(e, "attend: tensor-core kernel shared memory");
-    attr = true;
-  }
-  cudaError_t e = launch_pdl(attend_tc_kernel, dim3((unsigned)P.n_tiles, (unsigned)P.hkv, (unsigned)P.n_splits),
+  static std::atomic<uint64_t> attr{0};
+  cudaError_t e = smem_limit_once(attend_tc_kernel, kSmemTc, attr);
+  if (e != cudaSuccess) return cuda_fail(e, "attend: tensor-core kernel shared memory");
+  e = launch_pdl(attend_tc_kernel, dim3((unsigned)P.n_tiles, (unsigned)P.hkv, (unsigned)P.n_splits),
                              dim3(kThreadsTc),
                              (size_t)kSmemTc, st, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: tensor cores (many rows)");

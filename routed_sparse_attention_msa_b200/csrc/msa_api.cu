@@ -240,17 +240,17 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   p.doc_key = reinterpret_cast<uint32_t*>(w + L.doc_key);
   p.zero = w + L.doc_key;
   p.zero_bytes = L.total - L.doc_key;  // a multiple of 256
+  // automatic: many rows -> heads in turn with the scales in the epilogue
+  // (score_pf.cu), a few -> all heads' accumulators at once (score_tc.cu),
+  // other head counts -> CUDA cores
+  int which = g_score_kernel;
+  if (which == 0)
+    which = score_pf_supported(p) && n_rows > kManyRows ? 3 : score_tc_supported(p) ? 2 : 1;
+  if (b->n_chunks > 0 && ((which == 2 && !score_tc_supported(p)) || (which == 3 && !score_pf_supported(p))))
+    return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
   s = launch_qprep(p, eps, st);
   if (s != MSA_OK) return s;
   if (b->n_chunks > 0) {
-    // automatic: many rows -> heads in turn with the scales in the epilogue
-    // (score_pf.cu), a few -> all heads' accumulators at once (score_tc.cu),
-    // other head counts -> CUDA cores
-    int which = g_score_kernel;
-    if (which == 0)
-      which = score_pf_supported(p) && n_rows > kManyRows ? 3 : score_tc_supported(p) ? 2 : 1;
-    if ((which == 2 && !score_tc_supported(p)) || (which == 3 && !score_pf_supported(p)))
-      return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
     record_debug_event(0, st);
     s = which == 3 ? launch_score_pf(p, st) : which == 2 ? launch_score_tc(p, st) : launch_score_simt(p, st);
     record_debug_event(1, st);
@@ -447,7 +447,8 @@ msa_status msa_sync_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sync_check");
-  const int e_tc = tc_error_take(), e_pf = pf_error_take(), e_at = attend_tc_error_take(), e_pr = probe_error_take();
+  const int e_tc = tc_error_take(), e_pf = pf_error_take(), e_pr = probe_error_take();
+  const int e_at = attend_tc_error_take() | attend_dec_tc_error_take();
   if (e_tc || e_pf) return fail(MSA_ERR_TIMEOUT, "sync_check: a tensor-core scoring kernel gave up on a wait");
   if (e_pr) return fail(MSA_ERR_TIMEOUT, "sync_check: the wait probe's wait ran out");
   if (e_at) return fail(MSA_ERR_TIMEOUT, "sync_check: the tensor-core attention kernel gave up on a wait");

@@ -550,12 +550,10 @@ msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
   a.n_rows_pad = p.n_rows_pad;
   a.n_tiles = (int)((p.n_chunks + kM - 1) / kM);
   a.n_nb = (p.n_rows + NB - 1) / NB;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(score_pf_kernel<NB, WQ, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  static std::atomic<uint64_t> attr_set{0};
+  {
+    const cudaError_t e = smem_limit_once(score_pf_kernel<NB, WQ, PAIR>, C::kSmem, attr_set);
     if (e != cudaSuccess) return cuda_fail(e, "route: many-row scorer shared memory");
-    attr_set = true;
   }
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

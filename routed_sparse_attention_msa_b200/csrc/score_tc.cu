@@ -360,11 +360,10 @@ msa_status launch_nb(const RoutePlan& p, cudaStream_t st) {
   a.n_tiles = (int)((p.n_chunks + kTileM - 1) / kTileM);
   a.n_nb = (p.n_rows + NB - 1) / NB;
   for (int i = 0; i <= p.n_seq; ++i) a.q_seq_off[i] = p.q_seq_off[i];
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  static std::atomic<uint64_t> attr_set{0};
+  {
+    const cudaError_t e = smem_limit_once(score_tc_kernel<NB>, C::kSmem, attr_set);
     if (e != cudaSuccess) return cuda_fail(e, "route: tensor-core kernel shared memory");
-    attr_set = true;
   }
   int sms = 148;
   int dev = 0;

@@ -7,6 +7,9 @@ arguments returns MSA_ERR_CUDA (4) instead of the code tested here: each case
 below therefore also shows that the check comes before any CUDA work.
 """
 import ctypes
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -15,6 +18,22 @@ from tests.test_abi import load_build_module
 
 INVALID, WORKSPACE, UNSUPPORTED, CAPACITY = 1, 2, 3, 6
 FAKE = 0x1000  # a non-NULL pointer that is never dereferenced by the checks
+
+
+def _gpu_visible() -> bool:
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        return False
+
+
+# The cases below hand the library pointers that only the host checks keep
+# from reaching a kernel. In a process that can see a GPU they would run on
+# the device if a check ever moved, so there they are skipped and re-run as a
+# whole in a child process with no GPU visible (the last test of this file).
+_HOST_ONLY = os.environ.get("CUDA_VISIBLE_DEVICES") == "" or not _gpu_visible()
+host_only = pytest.mark.skipif(not _HOST_ONLY, reason="runs in a child process with no GPU visible")
 
 
 @pytest.fixture(scope="module")
@@ -64,6 +83,7 @@ ROUTE_CASES = [
 ]
 
 
+@host_only
 @pytest.mark.parametrize("bank_kw, call_kw, code, frag", ROUTE_CASES)
 def test_route_argument_checks(msa, bank_kw, call_kw, code, frag):
     b = _bank(msa, **bank_kw)
@@ -77,6 +97,7 @@ def test_route_argument_checks(msa, bank_kw, call_kw, code, frag):
     assert frag in _last(msa)
 
 
+@host_only
 def test_route_workspace_and_static_checks(msa):
     n = ctypes.c_size_t()
     b = _bank(msa)
@@ -97,6 +118,7 @@ def test_route_workspace_and_static_checks(msa):
 
 # ---------------------------------------------------------------- top-k merge
 
+@host_only
 def test_topk_merge_checks(msa):
     off = np.zeros(65, np.int64)
     f = msa._lib.msa_topk_merge
@@ -139,6 +161,7 @@ def _gather(msa, bank, **kw):
     (dict(content_on_host=1), dict(mode=0, done_event=None), INVALID, "copy-engine mode needs"),
     (dict(content_on_host=1), dict(mode=0, top_ids_host=None), INVALID, "copy-engine mode needs"),
 ])
+@host_only
 def test_gather_argument_checks(msa, bank_kw, call_kw, code, frag):
     b = _bank(msa, **bank_kw)
     g = _gather(msa, b, **call_kw)
@@ -186,6 +209,7 @@ ATTEND_CASES = [
 ]
 
 
+@host_only
 @pytest.mark.parametrize("kw, code, frag", ATTEND_CASES)
 def test_attend_argument_checks(msa, kw, code, frag):
     a, keep = _attend(msa, **dict(kw))
@@ -199,6 +223,7 @@ def test_attend_argument_checks(msa, kw, code, frag):
         assert frag in _last(msa)
 
 
+@host_only
 def test_attend_valid_arguments_need_a_workspace(msa):
     a, keep = _attend(msa)
     n = ctypes.c_size_t()
@@ -211,6 +236,7 @@ def test_attend_valid_arguments_need_a_workspace(msa):
     assert msa._lib.msa_attend(ctypes.byref(z), FAKE, 1 << 30, None) == 0
 
 
+@host_only
 def test_attend_backward_checks(msa):
     a, keep = _attend(msa)
     f = msa._lib.msa_attend_backward
@@ -248,6 +274,7 @@ def _encode(msa, **kw):
     (dict(rope_mode=2), INVALID, "rope_mode = 2"),
     (dict(kr_inv_norm=None), INVALID, "NULL tensor"),
 ])
+@host_only
 def test_encode_argument_checks(msa, kw, code, frag):
     e = _encode(msa, **kw)
     assert msa._lib.msa_encode(ctypes.byref(e), None) == code, _last(msa)
@@ -255,6 +282,7 @@ def test_encode_argument_checks(msa, kw, code, frag):
     assert msa._lib.msa_encode(None, None) == INVALID
 
 
+@host_only
 def test_bank_norms_and_route_backward_checks(msa):
     f = msa._lib.msa_bank_norms
     assert f(FAKE, 10, 8, 64, 1e-8, FAKE, None) == UNSUPPORTED
@@ -278,3 +306,12 @@ def test_bank_norms_and_route_backward_checks(msa):
     assert call(dqr=None) == INVALID and "NULL pointer" in _last(msa)
     empty = np.array([0, 0, 2], np.int32)
     assert call(qso=empty.ctypes.data, n_seq=2) == INVALID and "no rows" in _last(msa)
+
+
+@pytest.mark.skipif(_HOST_ONLY, reason="this process already runs the checks without a GPU")
+def test_argument_checks_in_a_process_without_gpu():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", os.path.abspath(__file__)],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]

@@ -41,6 +41,10 @@ def test_device_generator_matches_host():
     np.testing.assert_array_equal(bits(t), host_normal((1000,), synth.tid("kbar", 2), 0.5, 123456789))
 
 
+def bf16_of(x):
+    return synth.bf16_bits(np.asarray(x, np.float64))
+
+
 # ---------------------------------------------------------------- encode
 
 ENC_LENS = [64, 1, 63, 65, 0, 129, 300, 4096 + 17, 640, 2]
@@ -98,6 +102,39 @@ def test_bank_norms_match_oracle(msa):
     msa.bank_norms(z, inv, eps=1e-6)
     msa.sync_check()
     np.testing.assert_allclose(inv.cpu().numpy(), 1e6, rtol=1e-6)
+
+
+@pytest.mark.parametrize("chunk", [16, 128])
+def test_encode_other_chunk_lengths(msa, chunk):
+    """The chunk length is an argument: 16 and 128 against the oracle."""
+    lens = [chunk, 1, chunk - 1, chunk + 1, 0, 3 * chunk + 5]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    n = int(off[-1])
+    shp = (n, 8, 128)
+    k = dev_normal(shp, synth.tid("k_tok", 3))
+    v = dev_normal(shp, synth.tid("v_tok", 3))
+    r = dev_normal(shp, synth.tid("kr_tok", 3))
+    C, dco_h, mx = msa.encode_plan(off, chunk)
+    out = dict(kbar=torch.empty((C, 8, 128), dtype=torch.bfloat16, device="cuda"),
+               vbar=torch.empty((C, 8, 128), dtype=torch.bfloat16, device="cuda"),
+               kbar_r=torch.empty((C, 8, 128), dtype=torch.bfloat16, device="cuda"),
+               kr_inv_norm=torch.empty((C, 8), dtype=torch.float32, device="cuda"),
+               doc_chunk_off=torch.empty(len(lens) + 1, dtype=torch.int64, device="cuda"),
+               chunk_doc=torch.empty(C, dtype=torch.int32, device="cuda"))
+    msa.encode(k, v, r, torch.from_numpy(off).cuda(), C, out, chunk=chunk)
+    msa.sync_check()
+    ref = oracle.encode(host_normal(shp, synth.tid("k_tok", 3)), host_normal(shp, synth.tid("v_tok", 3)),
+                        host_normal(shp, synth.tid("kr_tok", 3)), off, chunk=chunk)
+    np.testing.assert_array_equal(out["doc_chunk_off"].cpu().numpy(), ref["doc_chunk_off"])
+    np.testing.assert_array_equal(out["chunk_doc"].cpu().numpy(), ref["chunk_doc"])
+    for name in ["kbar", "vbar", "kbar_r"]:
+        g = oracle.bf16_to_f64(bits(out[name]))
+        o = oracle.bf16_to_f64(ref[name])
+        # one bfloat16 ulp plus the fp32 accumulation error of a mean of <= chunk O(1) terms
+        tol = bf16_ulp(o) + chunk * 2.0 ** -24 * 4 + 1e-5
+        assert np.all(np.abs(g - o) <= tol), (name, float(np.abs(g - o).max()))
+        assert float(np.mean(g == o)) > 0.98, name
+    np.testing.assert_allclose(out["kr_inv_norm"].cpu().numpy(), ref["kr_inv_norm"], rtol=2e-4)
 
 
 # ----------------------------------------------------------------- route
@@ -209,6 +246,33 @@ def test_route_many_rows_each_block(msa, block, pair):
     np.testing.assert_allclose(alls[finite], o_all[finite], atol=1e-3, rtol=0)
 
 
+
+def test_route_norm_clamp_large_eps(msa, score_kernel):
+    """eps = 0.5: each norm is clamped separately, so short vectors score in
+    proportion to their length (the oracle's closed-form pin, on the GPU)."""
+    hr, d, D = 8, 128, 256
+    e = np.zeros((hr, d))
+    e[np.arange(hr), 3 * np.arange(hr)] = 1.0
+    kbar = np.stack([2.0 * e, 0.25 * e] + [np.roll(e, 1 + j % 2, axis=1) for j in range(D - 2)])
+    qr = np.stack([0.25 * e, 2.0 * e])
+    kb = bf16_of(kbar)
+    eps = 0.5
+    o_ids, o_sc, o_ds = oracle.route(kb, np.arange(D + 1), bf16_of(qr), [0, 1, 2], top_k=3, eps=eps)
+    kr = from_bits(kb)
+    inv = torch.empty((D, hr), dtype=torch.float32, device="cuda")
+    msa.bank_norms(kr, inv, eps=eps)
+    bank = msa.BankLayer(doc_chunk_off=torch.arange(D + 1, dtype=torch.int64, device="cuda"),
+                         chunk_doc=torch.arange(D, dtype=torch.int32, device="cuda"), kbar_r=kr, kr_inv_norm=inv)
+    ids = torch.empty((2, 3), dtype=torch.int32, device="cuda")
+    sc = torch.empty((2, 3), dtype=torch.float32, device="cuda")
+    ads = torch.empty((2, D), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(msa.route_workspace(bank, 2, 2, 3), dtype=torch.uint8, device="cuda")
+    msa.route(bank, from_bits(bf16_of(qr)), [0, 1, 2], 3, ids, sc, ws, all_doc_scores=ads, eps=eps)
+    msa.sync_check()
+    np.testing.assert_allclose(ads.cpu().numpy(), o_ds, atol=1e-6)
+    np.testing.assert_array_equal(ids.cpu().numpy(), o_ids)
+    np.testing.assert_allclose(sc.cpu().numpy()[:, :2], [[0.5, 0.25], [1.0, 0.5]], atol=1e-6)
+
 @pytest.mark.parametrize("n_docs", [900, 1800, 3500, 5000])
 def test_route_topk_paths(msa, n_docs):
     # the top-k's single-CTA variants (up to 1,024 / 2,048 / 4,096 documents) and the multi-CTA merge
@@ -302,7 +366,7 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc"])
+@pytest.fixture(params=["split", "tc", "tc_dec"])
 def attend_kernel(request, msa):
     old = msa.set_attend_kernel(request.param)
     yield request.param

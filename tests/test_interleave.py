@@ -11,12 +11,16 @@ torch = pytest.importorskip("torch")
 
 
 def _oracle_interleave(kr_host, dco, qr_bits, k, hops):
-    from routed_sparse_attention_msa_b200.interleave import next_document
+    """The interleave loop on the oracle. The generated id of a hop is the
+    best-ranked document of that hop's top-k not fetched before (written out
+    here, independently of the library's loop)."""
     fetched, per_hop, rows = [], [], qr_bits
     for _ in range(hops):
         ids, sc, ds = oracle.route(kr_host, dco, rows, [0, rows.shape[0]], k)
         per_hop.append((ids[0], ds[0]))
-        d = next_document(ids[0], set(fetched))
+        fresh = [int(x) for x in ids[0] if int(x) not in fetched]
+        assert fresh, "every top-k document already fetched"
+        d = fresh[0]
         fetched.append(d)
         rows = np.concatenate([rows, kr_host[dco[d]:dco[d + 1]]])
     return fetched, per_hop

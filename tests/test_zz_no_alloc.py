@@ -10,8 +10,6 @@ tolerance of the other routing tests (ids exact, scores within 1e-3).
 This file is collected last so that a run stopping at the first failure has
 already run every other test.
 """
-import ctypes
-
 import numpy as np
 import pytest
 
@@ -56,10 +54,22 @@ def test_route_static_matches_route_on_two_calls_in_a_row():
 
 
 def test_route_static_rejects_calls_beyond_its_scratch():
+    """A call whose scratch need exceeds the array is refused on the host with
+    MSA_ERR_CAPACITY. Every pointer is a real device buffer of the right size,
+    so the call would be valid (and in bounds) if the capacity check ever moved."""
     import routed_sparse_attention_msa_b200 as msa
-    # 2,000,000 documents need 8 MB of per-document scores: more than the 4 MiB scratch.
-    b = msa.BankLayerC(2_000_000, 2_000_000, 8, 8, 128, 1, 1, 1, 1, 1, 1, 1, 0, 0)
-    qso = np.array([0, 1], np.int32)
-    rc = msa._lib.msa_route_static(ctypes.byref(b), 1, qso.ctypes.data, 1, 1, 16, 1e-8, 1, 1, None, None)
-    assert rc == 6
-    assert "static scratch" in msa._lib.msa_last_error().decode()
+    # 256 sequences x 4,200 documents need 4.3 MB of per-document keys: more than the 4 MiB scratch.
+    n_docs, n_seq, k = 4200, 256, 16
+    bank = DevBank(np.arange(n_docs + 1, dtype=np.int64) * 64, 1, content=False)
+    need = msa.route_workspace(bank.layer_c, n_seq, n_seq, k)
+    assert need > msa.ROUTE_STATIC_SCRATCH_BYTES
+    qr = torch.zeros((n_seq, 8, 128), dtype=torch.bfloat16, device="cuda")
+    ids = torch.full((n_seq, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((n_seq, k), dtype=torch.float32, device="cuda")
+    qso = np.arange(n_seq + 1, dtype=np.int32)
+    with pytest.raises(msa.MsaError) as ei:
+        msa.route_static(bank.layer_c, qr, qso, k, ids, sc)
+    assert ei.value.code == 6  # MSA_ERR_CAPACITY
+    assert "static scratch" in str(ei.value)
+    msa.sync_check()
+    assert bool((ids == -1).all())  # nothing was enqueued
