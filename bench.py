@@ -199,8 +199,9 @@ class StageClock:
 
     STAGES = ("route", "gather", "attend")
 
-    def __init__(self, msa, torch):
+    def __init__(self, msa, torch, external=False):
         self._msa, self._torch = msa, torch
+        self._external = external  # event record nodes when captured in a CUDA graph
         self.marks = []  # (stage, start event, end event)
 
     def __getattr__(self, name):
@@ -209,8 +210,8 @@ class StageClock:
             return f
 
         def timed(*a, **k):
-            s = self._torch.cuda.Event(enable_timing=True)
-            e = self._torch.cuda.Event(enable_timing=True)
+            s = self._torch.cuda.Event(enable_timing=True, external=self._external)
+            e = self._torch.cuda.Event(enable_timing=True, external=self._external)
             s.record()
             f(*a, **k)
             e.record()
@@ -465,6 +466,30 @@ class Routed:
         self.torch.cuda.synchronize()
         return clock.per_call_us(reps * self.L)
 
+    def stage_times_graph(self, reps: int = 5) -> dict:
+        """Warm device time of each stage per layer inside a replayed CUDA graph
+        of the step: events recorded as graph nodes around every route, gather
+        and attend call, so host launch gaps are not counted. Median over
+        replays; 'step' is the whole replay between the first and last event."""
+        torch = self.torch
+        clock = StageClock(self.msa, torch, external=True)
+        real, self.msa = self.msa, clock
+        g = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                self.step()
+        finally:
+            self.msa = real
+        runs = []
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            r = clock.per_call_us(self.L)
+            r["step"] = 1e3 * clock.marks[0][1].elapsed_time(clock.marks[-1][2]) / self.L
+            runs.append(r)
+        del g
+        return {k: statistics.median(r[k] for r in runs) for k in runs[0]}
+
     def units_per_step(self) -> float:
         return float(self.w.memory_tokens) * self.S * self.L
 
@@ -477,6 +502,13 @@ class Routed:
     def score_bytes_per_launch(self) -> float:
         w = self.w
         return self.scored_chunks() * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+
+    def route_bytes_per_call(self) -> float:
+        """Algorithmic bytes of one msa_route call: the bank's routing keys,
+        inverse norms and chunk owners, the query rows, and the per-document
+        score keys written and read once by the top-k (4 B per document per
+        sequence each way)."""
+        return self.score_bytes_per_launch() + 2 * 4 * self.S * (self.dco.size - 1)
 
     def score_flops_per_launch(self) -> float:
         """The contraction: 2 flops per (query row, chunk, head, dimension)."""
@@ -797,6 +829,14 @@ def run_ours(args):
                               f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
 
     extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None, "mode": args.mode}
+    if w.name != "encode" and graph is not None and args.mode in ("decode", "train"):
+        # the routing call as a whole (query norms, scoring, top-k), warm, inside a replayed graph
+        st = eng.stage_times_graph()
+        extra["stage_us_per_layer_graph"] = st
+        rbytes = eng.route_bytes_per_call()
+        r_ach = rbytes / (st["route"] * 1e-6) / 1e9
+        roof["route_call"] = {"achieved": r_ach, "frac": r_ach / peak, "avg_call_us": st["route"],
+                              "algorithmic_bytes_per_call": rbytes, "unit": "GB/s", "peak": peak}
     if args.stage_times and w.name != "encode":
         extra["stage_us_per_layer"] = eng.stage_times()
     if args.mode == "sharded":

@@ -306,11 +306,14 @@ msa_status msa_gather(const msa_gather_args* args, void* stream);
  * NULL, mem_k[sel_off[s] + m], e.g. the staging buffer of msa_gather).
  * out is bf16 (nearest even of the fp32 result); out_f32 and lse are optional.
  * max_sel >= sel_off[s+1] - sel_off[s] for every s sizes the split-K grid.
- * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16, n_seq <= 256.
+ * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16, n_seq <= 256. q, k_loc,
+ * v_loc, mem_k, mem_v, out and out_f32 must be 16-byte aligned and the
+ * workspace 256-byte aligned (MSA_ERR_INVALID_ARG / MSA_ERR_WORKSPACE).
  * How it runs (not part of the contract): when a sequence's query vectors
  * (rows x hq / hkv) fill at least 64, the logits and P.V run on the tensor
- * cores (the logits at fp32 accuracy, P rounded to bf16); otherwise a split-K
- * decoding kernel on CUDA cores.
+ * cores (the logits at fp32 accuracy, P rounded to bf16); otherwise a
+ * decoding kernel on CUDA cores streams the key rows by cp.async, with
+ * memory and local keys in separate CTAs merged by log-sum-exp.
  * ---------------------------------------------------------------------- */
 typedef struct msa_attend_args {
   const uint16_t* q;          /* device [n_q, hq, d] bf16, not rotated */

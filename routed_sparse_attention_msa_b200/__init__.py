@@ -154,10 +154,11 @@ def score_events(begin, end) -> None:
 
 
 def set_attend_kernel(which: str) -> str:
-    """'auto', 'split' (split-K decoding kernel), 'tc' (tensor cores, many
-    rows) or 'tc_dec' (tensor cores with the keys as M, for decoding shapes);
-    returns the previous setting. Testing control."""
-    names = ["auto", "split", "tc", "tc_dec"]
+    """'auto', 'split' (split-K kernel), 'tc' (tensor cores, many rows),
+    'tc_dec' (tensor cores with the keys as M) or 'dec' (the decoding kernel
+    that 'auto' picks when a sequence's query vectors fill less than half a
+    128-vector tile); returns the previous setting. Testing control."""
+    names = ["auto", "split", "tc", "tc_dec", "dec"]
     return names[_lib.msa_debug_set_attend_kernel(names.index(which))]
 
 

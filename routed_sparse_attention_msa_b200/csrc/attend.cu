@@ -9,7 +9,8 @@
 //
 // Two kernels:
 //  1. rope_rows: rotates the query rows and the local keys once per call into
-//     fp32 copies, and clears the merge tickets. Each angle is formed and
+//     fp32 copies (local keys as bf16 high + low halves for the decoding kernel
+//     of attend_dec.cu), and clears the merge tickets. Each angle is formed and
 //     reduced modulo 2*pi in double, so positions of any size keep full
 //     accuracy, and then evaluated with sincosf.
 //  2. attend_split: split-K flash decoding. A CTA owns one kv head, a tile of
@@ -55,6 +56,14 @@ struct Smem {
 // together).
 constexpr int kRopeHeads = 4;
 
+// An angle (radians, double) reduced to [-pi, pi] in double, as a float: sincosf
+// then evaluates it on its short, accurate range for positions of any size.
+__device__ __forceinline__ float reduced_angle(double ang) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  return (float)(ang - two_pi * rint(ang * inv_two_pi));
+}
+
 __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
   pdl_wait();
   pdl_trigger();
@@ -80,10 +89,7 @@ __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
     const int s = seq_of(p.loc_off, p.n_seq, row);
     pos = p.pos_offset + (double)(row - p.loc_off[s]);
   }
-  const double w = exp2(-2.0 * (double)i / (double)kHeadDim * p.log2_theta);
-  const double ang = pos * w;
-  const double two_pi = 6.283185307179586476925286766559;
-  const float r = (float)(ang - two_pi * rint(ang / two_pi));  // in [-pi, pi]
+  const float r = reduced_angle(pos * p.inv_freq[i]);
   float sn, cs;
   sincosf(r, &sn, &cs);
   const size_t base = ((size_t)row * heads + h0) * kHeadDim + i;
@@ -99,8 +105,18 @@ __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
 #pragma unroll
   for (int u = 0; u < kRopeHeads; ++u) {
     if (h0 + u < heads) {
-      dst[u * kHeadDim] = x0[u] * cs - x1[u] * sn;
-      dst[u * kHeadDim + 64] = x0[u] * sn + x1[u] * cs;
+      const float y0 = x0[u] * cs - x1[u] * sn, y1 = x0[u] * sn + x1[u] * cs;
+      if (!is_q && p.krot_split) {  // bf16 high halves [0, 128), low halves [128, 256) of the row
+        uint16_t* kb = reinterpret_cast<uint16_t*>(p.krot) + ((size_t)row * heads + h0 + u) * 2 * kHeadDim;
+        const uint32_t b0 = f2bf_bits(y0), b1 = f2bf_bits(y1);
+        kb[i] = (uint16_t)b0;
+        kb[64 + i] = (uint16_t)b1;
+        kb[kHeadDim + i] = (uint16_t)f2bf_bits(y0 - __uint_as_float(b0 << 16));
+        kb[kHeadDim + 64 + i] = (uint16_t)f2bf_bits(y1 - __uint_as_float(b1 << 16));
+      } else {
+        dst[u * kHeadDim] = y0;
+        dst[u * kHeadDim + 64] = y1;
+      }
     }
   }
 }
@@ -370,11 +386,8 @@ __global__ void __launch_bounds__(kThreads) attend_split_kernel(const __grid_con
 // back (by the negative angle), pooled memory keys are used as stored.
 
 // Rotation of the pair (x, y) of dimension i by minus the angle at `pos`.
-__device__ __forceinline__ void rotate_back(float& x, float& y, int i, double pos, double log2_theta) {
-  const double w = exp2(-2.0 * (double)i / (double)kHeadDim * log2_theta);
-  const double ang = pos * w;
-  const double two_pi = 6.283185307179586476925286766559;
-  const float r = (float)(ang - two_pi * rint(ang / two_pi));
+__device__ __forceinline__ void rotate_back(float& x, float& y, int i, double pos, const double* inv_freq) {
+  const float r = reduced_angle(pos * inv_freq[i]);
   float sn, cs;
   sincosf(r, &sn, &cs);
   const float a = x * cs + y * sn;
@@ -552,7 +565,7 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_dq_kernel(const __grid_co
       const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
       float x = lane < 16 ? mine : other, y = lane < 16 ? other : mine;  // (dim, dim + 64)
       const int dim = 4 * (lane & 15) + e;
-      if (rr < nr) rotate_back(x, y, dim, p.pos_offset + (double)(g0 + rr), p.log2_theta);
+      if (rr < nr) rotate_back(x, y, dim, p.pos_offset + (double)(g0 + rr), p.inv_freq);
       o[e] = lane < 16 ? x : y;
     }
     if (rr < nr) {
@@ -681,7 +694,7 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_dkdv_kernel(const __grid_
     const float other = __shfl_xor_sync(0xffffffffu, ak[e], 2);
     if (local && jk < nb) {
       float x = (tid & 2) ? other : ak[e], y = (tid & 2) ? ak[e] : other;
-      rotate_back(x, y, (dsl & 63) + e, p.pos_offset + (double)(key - n_mem), p.log2_theta);
+      rotate_back(x, y, (dsl & 63) + e, p.pos_offset + (double)(key - n_mem), p.inv_freq);
       ak[e] = (tid & 2) ? y : x;
     }
   }
@@ -706,23 +719,26 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_dkdv_kernel(const __grid_
 
 struct Shape {
   int vec, rt, n_tiles, n_splits, n_loc;
-  bool tc;  // tensor-core kernel (many rows per sequence)
+  bool tc;   // tensor-core kernel (many rows per sequence)
+  bool dec;  // decoding kernel (attend_dec.cu)
 };
 
-int g_attend_kernel = 0;  // 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores (testing control)
+// 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores, 4 decoding
+// kernel on CUDA cores (testing control)
+int g_attend_kernel = 0;
 int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
 
 // allow_tc: the forward may take the tensor-core kernel when the query
 // vectors of a sequence fill at least half of its 128-vector tile.
 Shape plan(const msa_attend_args& a, bool allow_tc) {
-  Shape sh;
+  Shape sh{};
   const int group = a.hq / a.hkv;
   int max_rows = 1;
   for (int s = 0; s < a.n_seq; ++s) {
     const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
     max_rows = rows > max_rows ? rows : max_rows;
   }
-  sh.tc = allow_tc && g_attend_kernel != 1 && g_attend_kernel != 3 && kAttnTcVec % group == 0 &&
+  sh.tc = allow_tc && g_attend_kernel != 1 && g_attend_kernel != 3 && g_attend_kernel != 4 && kAttnTcVec % group == 0 &&
           (g_attend_kernel == 2 || max_rows * group >= kAttnTcVec / 2);
   if (sh.tc) {
     sh.vec = kAttnTcVec;
@@ -742,6 +758,7 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
     sh.n_splits = (int)std::max<int64_t>(splits, 1);
     return sh;
   }
+  sh.dec = allow_tc && (g_attend_kernel == 0 || g_attend_kernel == 4);
   // query vectors per CTA: the GQA group times enough rows, 4 to 16
   sh.vec = 4;
   while (sh.vec < kMaxVec && sh.vec < group * max_rows) sh.vec *= 2;
@@ -756,6 +773,23 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
     max_loc = max_loc > nl ? max_loc : nl;
   }
   sh.n_loc = a.loc_off[a.n_seq];
+  if (sh.dec) {
+    // one CTA per SM (the kernel takes ~165 KB of shared memory): key splits
+    // per (tile, kv head) while the grid is under 148 CTAs, each split an even
+    // share of the sequence's memory keys and of its local keys
+    int max_lvis = 0;
+    for (int s = 0; s < a.n_seq; ++s) {
+      const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
+      const int nl = a.loc_off[s + 1] - a.loc_off[s];
+      max_lvis = std::max(max_lvis, std::max(0, std::min(nl, a.q_start[s] + rows)));
+    }
+    const int64_t pairs = std::max<int64_t>((int64_t)sh.n_tiles * a.hkv, 1);
+    int64_t splits = g_attend_splits > 0 ? g_attend_splits : 148 / pairs;
+    const int64_t cap = (a.max_sel + max_lvis + 63) / 64;  // at least one 64-key block each
+    splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, cap), 64));
+    sh.n_splits = (int)splits;
+    return sh;
+  }
   const int64_t max_keys = a.max_sel + max_loc;
   const int64_t ctas = (int64_t)sh.n_tiles * a.hkv;
   int64_t splits = (2 * 148 + ctas - 1) / (ctas > 0 ? ctas : 1);
@@ -815,9 +849,11 @@ void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, cha
   P.out = a.out; P.out_f32 = a.out_f32; P.lse = a.lse;
   P.n_seq = a.n_seq; P.n_q = a.n_q; P.n_loc = sh.n_loc; P.hq = a.hq; P.hkv = a.hkv;
   P.group = a.hq / a.hkv; P.rt = sh.rt; P.n_splits = sh.n_splits; P.n_tiles = sh.n_tiles;
+  P.krot_split = sh.dec ? 1 : 0;
   P.scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)kHeadDim);
   P.pos_offset = (double)a.pos_offset;
   P.log2_theta = log2((double)a.rope_theta);
+  for (int i = 0; i < kHeadDim / 2; ++i) P.inv_freq[i] = exp2(-2.0 * (double)i / (double)kHeadDim * P.log2_theta);
   int t = 0;
   for (int s = 0; s < a.n_seq; ++s) {
     P.q_seq_off[s] = a.q_seq_off[s];
@@ -864,6 +900,7 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   if (s != MSA_OK) return s;
   if (sh.tc) return launch_attend_tc(P, st);
   if (g_attend_kernel == 3) return launch_attend_dec_tc(P, st);
+  if (sh.dec) return launch_attend_dec(P, sh.vec, st);
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
     case 4: return launch_vec<4>(P, grid, st);
@@ -919,11 +956,12 @@ msa_status launch_attend_backward(const msa_attend_args& a, const float* dout, f
 
 // Selects the attention kernel of later msa_attend calls in this process:
 // 0 = automatic, 1 = split-K, 2 = tensor cores (any row count), 3 = the
-// decoding tensor-core kernel (in place of split-K); returns the previous
-// setting. A testing and benchmarking control; not declared in msa.h.
+// decoding tensor-core kernel, 4 = the decoding kernel on CUDA cores (what
+// automatic picks for decoding shapes); returns the previous setting. A
+// testing and benchmarking control; not declared in msa.h.
 extern "C" int msa_debug_set_attend_kernel(int which) {
   const int old = msa::g_attend_kernel;
-  if (which >= 0 && which <= 3) msa::g_attend_kernel = which;
+  if (which >= 0 && which <= 4) msa::g_attend_kernel = which;
   return old;
 }
 

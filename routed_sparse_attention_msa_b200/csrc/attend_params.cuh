@@ -24,8 +24,10 @@ struct AttnParams {
   float* out_f32;
   float* lse;
   int n_seq, n_q, n_loc, hq, hkv, group, rt, n_splits, n_tiles;
+  int krot_split;  // 1: rope_rows stores each rotated local key as bf16 high halves then low halves (512 B)
   float scale;
   double pos_offset, log2_theta;
+  double inv_freq[kHeadDim / 2];  // RoPE frequency of pair i: theta^(-2i/d), formed on the host in double
   int32_t q_seq_off[kMaxSeq + 1];
   int32_t q_start[kMaxSeq];
   int32_t loc_off[kMaxSeq + 1];
@@ -52,6 +54,12 @@ int attend_tc_error_take();  // 1 if its bounded wait ran out since the last cal
 // the tensor cores, keys as the MMA's M side; same grid and split-K plan as
 // the split-K kernel. Needs rope_rows to have run.
 msa_status launch_attend_dec_tc(const AttnParams& P, cudaStream_t st);
+
+// attend_dec.cu: the decoding shapes (at most 16 query vectors per tile),
+// grid (n_splits, hkv, n_tiles), each split an even share of every
+// sequence's memory and local keys. Needs rope_rows to have run with
+// krot_split = 1.
+msa_status launch_attend_dec(const AttnParams& P, int vec, cudaStream_t st);
 int attend_dec_tc_error_take();
 
 }  // namespace msa

@@ -12,11 +12,17 @@ namespace msa {
 namespace {
 
 // One CTA: an exclusive scan over the (sequence, rank) pairs of the selected
-// documents' chunk counts gives each document's place in the list.
-__global__ void __launch_bounds__(1024) gather_index_kernel(
+// documents' chunk counts gives each document's place in the list; then all
+// threads write the list together, output position j taking its document by
+// a binary search over the scanned starts (coalesced stores, no per-document
+// loop).
+constexpr int kIndexThreads = 1024;
+
+__global__ void __launch_bounds__(kIndexThreads) gather_index_kernel(
     const int64_t* __restrict__ doc_chunk_off, const int32_t* __restrict__ top_ids, int n_seq,
     int k, int64_t* __restrict__ sel_off, int64_t* __restrict__ sel_chunk) {
   __shared__ int64_t warp_sums[32];
+  __shared__ int64_t s_start[kIndexThreads], s_c0[kIndexThreads];
   __shared__ int64_t carry;
   pdl_wait();
   pdl_trigger();
@@ -24,11 +30,11 @@ __global__ void __launch_bounds__(1024) gather_index_kernel(
   const int64_t n_pairs = (int64_t)n_seq * k;
   if (tid == 0) carry = 0;
   __syncthreads();
-  for (int64_t base = 0; base < n_pairs; base += blockDim.x) {
+  for (int64_t base = 0; base < n_pairs; base += kIndexThreads) {
     const int64_t p = base + tid;
     int64_t c0 = 0, n = 0;
     if (p < n_pairs) {
-      int32_t doc = top_ids[p];
+      const int32_t doc = __ldcg(top_ids + p);
       c0 = doc_chunk_off[doc];
       n = doc_chunk_off[doc + 1] - c0;
     }
@@ -41,7 +47,7 @@ __global__ void __launch_bounds__(1024) gather_index_kernel(
     if (lane == 31) warp_sums[wid] = x;
     __syncthreads();
     if (wid == 0) {
-      int64_t w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+      int64_t w = warp_sums[lane];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         int64_t y = __shfl_up_sync(0xffffffffu, w, o);
@@ -50,14 +56,26 @@ __global__ void __launch_bounds__(1024) gather_index_kernel(
       warp_sums[lane] = w;
     }
     __syncthreads();
-    const int64_t start = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + x - n;
+    const int64_t c_old = carry;
+    const int64_t start = c_old + (wid > 0 ? warp_sums[wid - 1] : 0) + x - n;
+    s_start[tid] = p < n_pairs ? start : INT64_MAX;
+    s_c0[tid] = c0;
     if (p < n_pairs) {
-      for (int64_t i = 0; i < n; ++i) sel_chunk[start + i] = c0 + i;
       if (p % k == 0) sel_off[p / k] = start;
       if (p == n_pairs - 1) sel_off[n_seq] = start + n;
     }
+    const int64_t c_new = c_old + warp_sums[31];
     __syncthreads();
-    if (tid == blockDim.x - 1) carry = start + n;
+    for (int64_t j = c_old + tid; j < c_new; j += kIndexThreads) {
+      int lo = 0, hi = kIndexThreads - 1;  // the last pair whose start is <= j
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_start[mid] <= j) lo = mid; else hi = mid - 1;
+      }
+      sel_chunk[j] = s_c0[lo] + (j - s_start[lo]);
+    }
+    __syncthreads();
+    if (tid == 0) carry = c_new;
     __syncthreads();
   }
 }

@@ -375,6 +375,10 @@ static msa_status check_attend(const msa_attend_args* a) {
   if (a->max_sel < 0) return fail(MSA_ERR_INVALID_ARG, "attend: max_sel < 0");
   if (a->max_sel > 0 && (!a->mem_k || !a->mem_v)) return fail(MSA_ERR_INVALID_ARG, "attend: NULL memory K/V");
   if (!(a->rope_theta > 1.0f)) return fail(MSA_ERR_INVALID_ARG, "attend: rope_theta must be > 1");
+  // the kernels move rows in 16-byte pieces
+  const void* rows[] = {a->q, a->k_loc, a->v_loc, a->mem_k, a->mem_v, a->out, a->out_f32};
+  for (const void* r : rows)
+    if (reinterpret_cast<uintptr_t>(r) & 15) return fail(MSA_ERR_INVALID_ARG, "attend: row arrays must be 16-byte aligned");
   return MSA_OK;
 }
 
@@ -391,6 +395,7 @@ msa_status msa_attend(const msa_attend_args* a, void* ws, size_t ws_bytes, void*
   if (s != MSA_OK) return s;
   size_t need = attend_workspace(*a, nullptr);
   if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "attend: workspace %zu B, need %zu B", ws_bytes, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(MSA_ERR_WORKSPACE, "attend: workspace must be 256-byte aligned");
   if (a->n_q == 0) return MSA_OK;
   return launch_attend(*a, ws, (cudaStream_t)stream);
 }

@@ -129,7 +129,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // the prologue above overlapped the previous kernel's tail
+  // The producer and the MMA warp read only the bank and the query rows, which
+  // are inputs of the call and complete before the preceding kernel (the query
+  // preparation) started; they begin streaming at once, overlapping that
+  // kernel. The epilogue reads its outputs (query scales, the cleared document
+  // keys) and waits for it first.
+  if (warp >= kEpiWarp0) pdl_wait();
   pdl_trigger();
 
   if (warp == 0) {

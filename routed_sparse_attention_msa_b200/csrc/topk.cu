@@ -10,14 +10,15 @@
 // has score word 0, below every real score.
 //
 // k <= 16: each warp keeps its best 16 keys sorted across lanes 0..15 (up to
-// 4,096 documents: one CTA per sequence, no cross-CTA merge). A batch
+// 2,048 documents: one CTA per sequence, no cross-CTA merge). A batch
 // of 32 new keys is first tested against the 16th key with one ballot (after
 // the first batches almost every batch is skipped); otherwise the batch is
 // sorted by a 32-lane bitonic network and merged with the list by one
 // bitonic merge (the list in lanes 0..15, the batch's best 16 reversed into
-// lanes 16..31). Warps, then CTAs, are combined by the same merge. The last
-// CTA of a sequence to finish (atomic ticket, no waiting) merges the CTAs'
-// lists. 16 < k <= 32: the same structure with per-key insertion by shuffles.
+// lanes 16..31). Warps (as a tree), then CTAs, are combined by the same
+// merge. Beyond 2,048 documents a sequence is split into CTAs of 2,048 and
+// the last CTA of the sequence to finish (atomic ticket, no waiting) merges
+// the CTAs' lists. 16 < k <= 32: the same structure with per-key insertion by shuffles.
 // k > 32: one CTA per sequence runs an 8-pass radix select on the keys,
 // collects the k keys at or above the k-th and sorts them.
 #include "msa_internal.cuh"
@@ -148,15 +149,41 @@ __global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(
   if (lane == 0) tickets[s] = 0u;  // ready for the next call
 }
 
-// IT batches of 32 keys per warp (kWarps * 32 * IT documents per CTA). With
-// one CTA per sequence the result is written directly, without the
-// candidate lists and the ticket.
+// k <= 16, 32 warps per CTA: IT batches of 32 keys per warp (1,024 * IT
+// documents per CTA), every key load issued before any merging. The warps'
+// lists are combined by a 5-level tree of merges in shared memory. With one
+// CTA per sequence (up to 2,048 documents) the result is written directly;
+// otherwise each CTA writes its list and the last CTA of the sequence to
+// finish (atomic ticket, no waiting) merges them.
+constexpr int kWarps16 = 32;
+// Measured on 16 sequences x 10,040 documents: one CTA per sequence (16 batches
+// per warp) 20 us, CTAs of 1,024 documents with the last-CTA merge 10.6 us; the
+// batches of a warp are a dependent chain, so documents are spread over CTAs.
+constexpr int kSinglePassDocs = 2 * 1024;  // one CTA per sequence up to this many documents
+constexpr int kPartDocs = 2 * 1024;        // documents per CTA beyond it
+
+__device__ __forceinline__ uint64_t tree_merge16(uint64_t (*lists)[16], uint64_t list, int lane, int wid) {
+  // lists[w] holds warp w's best 16 (lanes 0..15 of `list` on entry); returns the overall best 16 in warp 0
+  if (lane < 16) lists[wid][lane] = list;
+  __syncthreads();
+#pragma unroll
+  for (int half = kWarps16 / 2; half > 0; half >>= 1) {
+    if (wid < half) {
+      list = warp_merge16(lane < 16 ? lists[wid][lane] : 0ull, lane < 16 ? lists[wid + half][lane] : 0ull, lane);
+      __syncwarp();
+      if (lane < 16) lists[wid][lane] = list;
+    }
+    __syncthreads();
+  }
+  return lane < 16 ? lists[0][lane] : 0ull;
+}
+
 template <int IT>
-__global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
+__global__ void __launch_bounds__(kWarps16 * 32) topk16_kernel(
     const uint32_t* __restrict__ doc_key, int64_t n_docs, int k, uint64_t* __restrict__ cand,
     unsigned* __restrict__ tickets, int32_t* __restrict__ top_ids, float* __restrict__ top_scores,
     float* __restrict__ all_scores) {
-  __shared__ uint64_t s_lists[kWarps][16];
+  __shared__ uint64_t s_lists[kWarps16][16];
   __shared__ bool s_last;
   pdl_wait();
   pdl_trigger();
@@ -166,15 +193,15 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
   const int n_parts = gridDim.x;
   const uint32_t* keys = doc_key + (size_t)s * n_docs;
 
-  // keys of this warp's slice, all loads issued before any merging
-  const int64_t w0 = (int64_t)part * (kWarps * 32 * IT) + (int64_t)wid * (32 * IT);
+  // keys of this warp's slice: document w0 + 32 it + lane
+  const int64_t w0 = (int64_t)part * (kWarps16 * 32 * IT) + (int64_t)wid * (32 * IT);
   uint64_t kv[IT];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const int64_t doc = w0 + it * 32 + lane;
     kv[it] = 0;
     if (doc < n_docs) {
-      const uint32_t sk = keys[doc];
+      const uint32_t sk = __ldcg(keys + doc);
       kv[it] = doc_key64(sk, doc);
       if (all_scores) all_scores[(size_t)s * n_docs + doc] = unord_f32(sk);
     }
@@ -182,16 +209,12 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
   uint64_t list = warp_sort32_desc(kv[0], lane);
 #pragma unroll
   for (int it = 1; it < IT; ++it) warp_fold32(list, kv[it], lane);
-  if (lane < 16) s_lists[wid][lane] = list;
-  __syncthreads();
+  uint64_t merged = tree_merge16(s_lists, list, lane, wid);
+  if (n_parts == 1) {  // the whole sequence in this CTA
+    if (wid == 0 && lane < k) write_result(merged, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
+    return;
+  }
   if (wid == 0) {
-    uint64_t merged = lane < 16 ? s_lists[0][lane] : 0ull;
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) merged = warp_merge16(merged, lane < 16 ? s_lists[w][lane] : 0ull, lane);
-    if (n_parts == 1) {  // the whole sequence in this CTA
-      if (lane < k) write_result(merged, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
-      return;
-    }
     if (lane < 16) cand[((size_t)s * n_parts + part) * 16 + lane] = merged;
     __threadfence();
     unsigned t = 0;
@@ -202,19 +225,20 @@ __global__ void __launch_bounds__(kWarps * 32) topk16_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // last CTA: every warp merges a share of the CTAs' lists, then warp 0 merges the warps'
+  // last CTA: every warp merges a share of the CTAs' lists, then the tree merges the warps'
   const uint64_t* c = cand + (size_t)s * n_parts * 16;
   uint64_t acc = 0;
-  for (int pp = wid; pp < n_parts; pp += kWarps)
+  for (int pp = wid; pp < n_parts; pp += kWarps16)
     acc = warp_merge16(acc, lane < 16 ? __ldcg(c + (size_t)pp * 16 + lane) : 0ull, lane);
-  if (lane < 16) s_lists[wid][lane] = acc;
-  __syncthreads();
-  if (wid != 0) return;
-  uint64_t fin = lane < 16 ? s_lists[0][lane] : 0ull;
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) fin = warp_merge16(fin, lane < 16 ? s_lists[w][lane] : 0ull, lane);
-  if (lane < k) write_result(fin, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
-  if (lane == 0) tickets[s] = 0u;  // ready for the next call
+  const uint64_t fin = tree_merge16(s_lists, acc, lane, wid);
+  if (wid == 0) {
+    if (lane < k) write_result(fin, top_ids + (size_t)s * k + lane, top_scores + (size_t)s * k + lane);
+    if (lane == 0) tickets[s] = 0u;  // ready for the next call
+  }
+}
+
+int topk16_parts(int64_t n_docs) {
+  return n_docs <= kSinglePassDocs ? 1 : (int)((n_docs + kPartDocs - 1) / kPartDocs);
 }
 
 // Generic path: one CTA (1024 threads) per sequence.
@@ -375,7 +399,7 @@ msa_status launch_topk_merge(const int32_t* ids, const float* scores, const int6
 }
 
 size_t topk_workspace(int n_seq, int64_t n_docs, int k) {
-  int64_t parts = (n_docs + kDocsPerCta - 1) / kDocsPerCta;
+  int64_t parts = k <= 16 ? topk16_parts(n_docs) : (n_docs + kDocsPerCta - 1) / kDocsPerCta;
   if (k > 32) return 256;
   const int kc = k <= 16 ? 16 : k;
   return align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256) +
@@ -393,21 +417,29 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
     unsigned* tickets = reinterpret_cast<unsigned*>(
         reinterpret_cast<char*>(ws) + align_up((size_t)n_seq * parts * kc * sizeof(uint64_t), 256));
     cudaError_t e;
-    if (k <= 16 && n_docs <= 4 * kDocsPerCta) {  // one CTA per sequence
-      const dim3 grid(1u, (unsigned)n_seq);
-      if (n_docs <= kDocsPerCta)
-        e = launch_pdl(topk16_kernel<kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k, cand,
-                       tickets, top_ids, top_scores, all_scores);
-      else if (n_docs <= 2 * kDocsPerCta)
-        e = launch_pdl(topk16_kernel<2 * kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k,
-                       cand, tickets, top_ids, top_scores, all_scores);
-      else
-        e = launch_pdl(topk16_kernel<4 * kDocsPerWarp / 32>, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k,
-                       cand, tickets, top_ids, top_scores, all_scores);
+    if (k <= 16) {
+      parts = topk16_parts(n_docs);
+      cand = reinterpret_cast<uint64_t*>(ws);
+      tickets = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(ws) +
+                                            align_up((size_t)n_seq * parts * 16 * sizeof(uint64_t), 256));
+      const dim3 grid((unsigned)parts, (unsigned)n_seq);
+      const int64_t per_cta = parts == 1 ? n_docs : kPartDocs;  // documents one CTA covers
+      const int it = per_cta <= 1024 ? 1 : per_cta <= 2048 ? 2 : per_cta <= 4096 ? 4 : per_cta <= 8192 ? 8 : 16;
+      auto go = [&](auto kernel) {
+        return launch_pdl(kernel, grid, dim3(kWarps16 * 32), 0, st, doc_key, n_docs, k, cand, tickets, top_ids,
+                          top_scores, all_scores);
+      };
+      switch (it) {
+        case 1: e = go(topk16_kernel<1>); break;
+        case 2: e = go(topk16_kernel<2>); break;
+        case 4: e = go(topk16_kernel<4>); break;
+        case 8: e = go(topk16_kernel<8>); break;
+        default: e = go(topk16_kernel<16>); break;
+      }
     } else {
       const dim3 grid((unsigned)parts, (unsigned)n_seq);
-      e = launch_pdl(k <= 16 ? topk16_kernel<kDocsPerWarp / 32> : topk_warp_kernel, grid, dim3(kWarps * 32), 0, st,
-                     doc_key, n_docs, k, cand, tickets, top_ids, top_scores, all_scores);
+      e = launch_pdl(topk_warp_kernel, grid, dim3(kWarps * 32), 0, st, doc_key, n_docs, k, cand, tickets, top_ids,
+                     top_scores, all_scores);
     }
     if (e != cudaSuccess) return cuda_fail(e, "route: top-k");
     return launch_check("route: top-k");

@@ -16,7 +16,7 @@ import bench  # noqa: E402
 class _FakeEvent:
     clock = 0.0
 
-    def __init__(self, enable_timing=False):
+    def __init__(self, enable_timing=False, external=False):
         self.t = None
 
     def record(self, stream=None):

@@ -273,9 +273,10 @@ def test_route_norm_clamp_large_eps(msa, score_kernel):
     np.testing.assert_array_equal(ids.cpu().numpy(), o_ids)
     np.testing.assert_allclose(sc.cpu().numpy()[:, :2], [[0.5, 0.25], [1.0, 0.5]], atol=1e-6)
 
-@pytest.mark.parametrize("n_docs", [900, 1800, 3500, 5000])
+@pytest.mark.parametrize("n_docs", [900, 1800, 3500, 5000, 12000, 20000, 41000])
 def test_route_topk_paths(msa, n_docs):
-    # the top-k's single-CTA variants (up to 1,024 / 2,048 / 4,096 documents) and the multi-CTA merge
+    # the top-k's single-CTA variant (up to 2,048 documents) and the multi-CTA merge (2,048 documents
+    # per CTA: 2 to 21 CTAs per sequence)
     off = _ragged_offsets(17 + n_docs, n_docs)
     bank = DevBank(off, 8, content=False)
     rows = (1, 3)
@@ -366,7 +367,7 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc", "tc_dec"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec"])
 def attend_kernel(request, msa):
     old = msa.set_attend_kernel(request.param)
     yield request.param
@@ -452,11 +453,14 @@ def test_attend_staged_memory_equals_indexed(msa, attend_kernel):
     np.testing.assert_array_equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("kernel", ["split", "dec"])
 @pytest.mark.parametrize("splits", [1, 2, 5, 64])
-def test_attend_forced_splits(msa, splits):
-    """The split-K kernel with its key-split count forced (64 is clamped to one
-    split per 32 keys): splits that get no keys, one split, uneven splits."""
-    old_k, old_s = msa.set_attend_kernel("split"), msa.set_attend_splits(splits)
+def test_attend_forced_splits(msa, kernel, splits):
+    """Key splits forced (split-K: 64 is clamped to one split per 32 keys;
+    decoding kernel: the memory-key CTAs, at least 64 keys each, so one or two
+    splits walk several pipelined blocks): splits that get no keys, one split,
+    uneven splits."""
+    old_k, old_s = msa.set_attend_kernel(kernel), msa.set_attend_splits(splits)
     try:
         c = _attend_case(rows=(1, 1, 2), n_loc=(65, 1, 9), n_mem=(0, 300, 61), q_start=(64, 0, 7), layer=23)
         g_out, g_f32, g_lse = _attend_gpu(msa, c, 16.0)

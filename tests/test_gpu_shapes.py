@@ -124,7 +124,7 @@ def test_gather_host_tier_head_counts(msa, hkv):
 
 # ----------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc", "tc_dec"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec"])
 def attend_kernel(request, msa):
     old = msa.set_attend_kernel(request.param)
     yield request.param
