@@ -56,9 +56,10 @@ def parse_args():
     p.add_argument("--seqs", type=int, default=0, help="override the workload's sequence count (0: as defined)")
     p.add_argument("--mode", choices=["decode", "train", "sharded", "interleave"], default="decode",
                    help="decode: the routed decode step (default); train: decode step plus the gradients of "
-                        "attention and of the routing scores; sharded: routing of every layer split into "
-                        "--shards document shards merged by the top-k merge (Memory Parallel, emulated on one "
-                        "GPU); interleave: --hops routing hops per layer (Memory Interleave)")
+                        "attention and of the routing scores; sharded: Memory Parallel routing, every layer's "
+                        "bank split into document shards merged by the top-k merge (on one GPU: --shards shards "
+                        "one after another; under torchrun: one shard per rank, candidates all-gathered over "
+                        "NCCL); interleave: --hops routing hops per layer (Memory Interleave)")
     p.add_argument("--prefill", action="store_true",
                    help="time the prefill step instead: every sequence routes and attends with its prefill rows "
                         "(1m: 128, 10m: 64 per sequence), causal over those rows")
@@ -245,17 +246,30 @@ class Routed:
         S, k = w.n_seq, w.top_k
         self.S, self.k = S, k
         hr, hkv, d = w.hr, w.hkv, w.d
+        # Memory Parallel across ranks: this rank holds one contiguous document
+        # shard of every layer's routing keys and routes only that
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.mp_ranks = args.mode == "sharded" and self.world > 1
+        r0 = 0
+        if self.mp_ranks:
+            from routed_sparse_attention_msa_b200 import memory_parallel as mp
+            self.mp = mp
+            self.rank_ranges = mp.shard_ranges(self.dco, self.world)
+            d0, d1 = self.rank_ranges[self.rank]
+            r0, r1 = int(self.dco[d0]), int(self.dco[d1])
+        n_rows_kr = (r1 - r0) if self.mp_ranks else self.C
 
-        def dev_normal(shape, tid):
+        def dev_normal(shape, tid, index0=0):
             t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
-            synth.normal_bf16_device(t.data_ptr(), t.numel(), tid, stream=st)
+            synth.normal_bf16_device(t.data_ptr(), t.numel(), tid, index0, stream=st)
             return t
 
-        # routing-key banks, one per layer, resident in HBM
+        # routing-key banks, one per layer, resident in HBM (this rank's shard of them)
         self.kbar_r, self.inv = [], []
         for l in range(self.L):
-            kr = dev_normal((self.C, hr, d), synth.tid("kbar_r", l))
-            iv = torch.empty((self.C, hr), dtype=torch.float32, device="cuda")
+            kr = dev_normal((n_rows_kr, hr, d), synth.tid("kbar_r", l), r0 * hr * d)
+            iv = torch.empty((n_rows_kr, hr), dtype=torch.float32, device="cuda")
             msa.bank_norms(kr, iv)
             self.kbar_r.append(kr)
             self.inv.append(iv)
@@ -275,9 +289,17 @@ class Routed:
                 self.kbar.append(dev_normal((self.C, hkv, d), synth.tid("kbar", l)))
                 self.vbar.append(dev_normal((self.C, hkv, d), synth.tid("vbar", l)))
         self.n_content = n_content
+        # with a routing-key shard, these banks serve the gather (document offsets and content only)
         self.banks = [msa.BankLayer(self.dco_d, self.cdoc_d, self.kbar_r[l], self.inv[l],
                                     self.kbar[l % n_content], self.vbar[l % n_content], self.on_host,
                                     self.max_doc_chunks) for l in range(self.L)]
+        if self.mp_ranks:
+            local_dco = torch.from_numpy(self.dco[d0:d1 + 1] - r0).cuda()
+            nch = np.diff(self.dco[d0:d1 + 1])
+            local_cdoc = torch.from_numpy(np.repeat(np.arange(d1 - d0, dtype=np.int32), nch)).cuda()
+            self.rank_shards = [mp.Shard(msa.BankLayer(local_dco, local_cdoc, self.kbar_r[l], self.inv[l], None, None,
+                                                       False, int(nch.max()) if nch.size else 0), d0, d1)
+                                for l in range(self.L)]
         # per-layer query routing rows with planted documents (built on the host)
         rows = [w.route_rows] * S
         self.T = sum(rows)
@@ -323,7 +345,9 @@ class Routed:
         self.scores_all = torch.empty((self.L, S, kk), dtype=torch.float32, device="cuda")
         self.ids = [self.ids_all[l] for l in range(self.L)]
         self.scores = [self.scores_all[l] for l in range(self.L)]
-        self.ws_route = torch.empty(msa.route_workspace(self.banks[0], S, self.T, k), dtype=torch.uint8, device="cuda")
+        route_bank0 = self.rank_shards[0].layer if self.mp_ranks else self.banks[0]
+        self.ws_route = torch.empty(max(msa.route_workspace(route_bank0, S, self.T, k), 256), dtype=torch.uint8,
+                                    device="cuda")
         self.cap = S * kk * self.max_doc_chunks
         self.sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
         self.sel = torch.empty(self.cap, dtype=torch.int64, device="cuda")
@@ -346,7 +370,7 @@ class Routed:
             raise SystemExit("--mode interleave follows one sequence; use a workload with one sequence")
         if args.mode == "train":
             self._setup_train(a0)
-        elif args.mode == "sharded":
+        elif args.mode == "sharded" and not self.mp_ranks:
             self._setup_sharded(args.shards)
         torch.cuda.synchronize()
 
@@ -406,7 +430,15 @@ class Routed:
 
     def layer(self, l, ev=None):
         msa = self.msa
-        if self.run_mode == "sharded":
+        if self.mp_ranks:
+            # Memory Parallel across ranks: route this rank's shard, all-gather every
+            # rank's candidates (NCCL), merge into the global top-k on every rank
+            if ev is not None:
+                msa.score_events(ev[0], ev[1])
+            self.mp.route_memory_parallel(self.rank_shards[l], [a for a, _ in self.rank_ranges], self.qr_d[l],
+                                          self.qso, self.k, self.ids[l], self.scores[l], self.ws_route,
+                                          eps=self.w.eps)
+        elif self.run_mode == "sharded":
             # Memory Parallel, one shard after another: route every shard, merge
             for g, sh in enumerate(self.shards[l]):
                 if g == 0 and ev is not None:
@@ -491,9 +523,15 @@ class Routed:
         return {k: statistics.median(r[k] for r in runs) for k in runs[0]}
 
     def units_per_step(self) -> float:
-        return float(self.w.memory_tokens) * self.S * self.L
+        """This rank's share of the step's memory tokens routed: the whole bank per
+        replica, or 1/world of it when the ranks split the bank (Memory Parallel)."""
+        full = float(self.w.memory_tokens) * self.S * self.L
+        return full / self.world if self.mp_ranks else full
 
     def scored_chunks(self) -> int:
+        if self.mp_ranks:  # this rank's shard
+            d0, d1 = self.rank_ranges[self.rank]
+            return int(self.dco[d1] - self.dco[d0])
         if self.run_mode == "sharded":  # the timed launch is shard 0's
             d0, d1 = self.shard_ranges[0]
             return int(self.dco[d1] - self.dco[d0])
@@ -728,7 +766,8 @@ def run_ours(args):
         planted_ok = bad == 0
 
     # ---- timed region: K steps, inputs resident in HBM
-    use_graph = args.graph == "on" or (args.graph == "auto" and args.mode != "interleave" and not (
+    mp_ranks = getattr(eng, "mp_ranks", False)
+    use_graph = args.graph == "on" or (args.graph == "auto" and args.mode != "interleave" and not mp_ranks and not (
         w.name != "encode" and w.content_on_host and args.gather == "copy"))
     graph = None
     if use_graph:
@@ -850,9 +889,11 @@ def run_ours(args):
     if w.name != "encode" and w.content_on_host:
         extra["host_content_banks"] = eng.n_content
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if mp_ranks else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, eng, args, extra), "parallelism": f"replicas{world}",
+            "config": config_of(w, eng, args, extra),
+            "parallelism": f"memory_parallel{world}" if mp_ranks else f"replicas{world}",
             "e2e": e2e, "gpu_launches": launches, "roofline": roof, "cpu_baseline": cpu,
             "clocks": clk.summary()}
     if rank == 0:

@@ -83,15 +83,24 @@ def route_local(shard: Shard, qr, q_seq_off_host, top_k: int, ids_out, scores_ou
 
 
 def gather_candidates(ids, scores, group=None):
-    """All-gather every rank's [S, k] candidates into [G, S, k] (torch.distributed)."""
+    """All-gather every rank's [S, k] candidates into [G, S, k] (torch.distributed).
+    NCCL gathers the device tensors directly (over NVLink); a gloo group gathers
+    host copies, and the result is returned on the candidates' device."""
     import torch
     import torch.distributed as dist
     G = dist.get_world_size(group)
-    li = [torch.empty_like(ids) for _ in range(G)]
-    ls = [torch.empty_like(scores) for _ in range(G)]
-    dist.all_gather(li, ids.contiguous(), group=group)
-    dist.all_gather(ls, scores.contiguous(), group=group)
-    return torch.stack(li), torch.stack(ls)
+    dev = ids.device
+    staged = dist.get_backend(group) == "gloo" and dev.type == "cuda"
+    src_i = ids.contiguous().cpu() if staged else ids.contiguous()
+    src_s = scores.contiguous().cpu() if staged else scores.contiguous()
+    li = [torch.empty_like(src_i) for _ in range(G)]
+    ls = [torch.empty_like(src_s) for _ in range(G)]
+    dist.all_gather(li, src_i, group=group)
+    dist.all_gather(ls, src_s, group=group)
+    all_i, all_s = torch.stack(li), torch.stack(ls)
+    if staged:
+        all_i, all_s = all_i.to(dev), all_s.to(dev)
+    return all_i, all_s
 
 
 def route_memory_parallel(shard: Shard, doc_offsets: list[int], qr, q_seq_off_host, top_k: int, top_ids,
