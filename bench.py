@@ -49,17 +49,20 @@ def parse_args():
                    help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
-    p.add_argument("--content-layers", type=int, default=1,
-                   help="host-tier content banks to allocate; layer l uses bank l mod this (0: one per layer "
-                        "if host RAM allows)")
+    p.add_argument("--content-layers", type=int, default=0,
+                   help="host-tier content banks to allocate; layer l uses bank l mod this (0, the default: one "
+                        "per layer if host RAM allows, else one shared by all layers)")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count (0: as defined)")
     p.add_argument("--seqs", type=int, default=0, help="override the workload's sequence count (0: as defined)")
-    p.add_argument("--mode", choices=["decode", "train", "sharded", "interleave"], default="decode",
+    p.add_argument("--gen-steps", type=int, default=64, help="--mode generate: tokens decoded after the prefill")
+    p.add_argument("--mode", choices=["decode", "train", "sharded", "interleave", "generate"], default="decode",
                    help="decode: the routed decode step (default); train: decode step plus the gradients of "
                         "attention and of the routing scores; sharded: Memory Parallel routing, every layer's "
                         "bank split into document shards merged by the top-k merge (on one GPU: --shards shards "
                         "one after another; under torchrun: one shard per rank, candidates all-gathered over "
-                        "NCCL); interleave: --hops routing hops per layer (Memory Interleave)")
+                        "NCCL); interleave: --hops routing hops per layer (Memory Interleave); generate: "
+                        "the prefill step then --gen-steps routed decoding steps with a growing local context, "
+                        "one CUDA graph per generated sequence")
     p.add_argument("--prefill", action="store_true",
                    help="time the prefill step instead: every sequence routes and attends with its prefill rows "
                         "(1m: 128, 10m: 64 per sequence), causal over those rows")
@@ -68,6 +71,8 @@ def parse_args():
     p.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
                    help="replay each step as one CUDA graph (auto: on unless the copy-engine gather needs host syncs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-cpu-all-cores", action="store_true",
+                   help="skip the all-core run of the CPU baseline (one oracle process per core)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--stage-times", action="store_true",
                    help="after the timed region, time route / gather / attend separately (CUDA events around "
@@ -220,9 +225,14 @@ class StageClock:
         return timed
 
     def per_call_us(self, calls: int) -> dict:
-        tot = {}
+        """Device time per call of each stage: the stage's total over `calls`
+        calls (calls <= 0: over the number of calls recorded for it)."""
+        tot, cnt = {}, {}
         for name, s, e in self.marks:
             tot[name] = tot.get(name, 0.0) + 1e3 * s.elapsed_time(e)
+            cnt[name] = cnt.get(name, 0) + 1
+        if calls <= 0:
+            return {k: v / cnt[k] for k, v in tot.items()}
         return {k: v / calls for k, v in tot.items()}
 
 
@@ -516,7 +526,7 @@ class Routed:
         for _ in range(reps):
             g.replay()
             torch.cuda.synchronize()
-            r = clock.per_call_us(self.L)
+            r = clock.per_call_us(0)  # per call of each stage
             r["step"] = 1e3 * clock.marks[0][1].elapsed_time(clock.marks[-1][2]) / self.L
             runs.append(r)
         del g
@@ -537,9 +547,13 @@ class Routed:
             return int(self.dco[d1] - self.dco[d0])
         return self.C
 
+    def timed_rows(self) -> int:
+        """Query rows of the scoring launch the roofline times."""
+        return self.T
+
     def score_bytes_per_launch(self) -> float:
         w = self.w
-        return self.scored_chunks() * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.T * w.hr * w.d * 2
+        return self.scored_chunks() * (w.hr * w.d * 2 + w.hr * 4 + 4) + self.timed_rows() * w.hr * w.d * 2
 
     def route_bytes_per_call(self) -> float:
         """Algorithmic bytes of one msa_route call: the bank's routing keys,
@@ -551,7 +565,7 @@ class Routed:
     def score_flops_per_launch(self) -> float:
         """The contraction: 2 flops per (query row, chunk, head, dimension)."""
         w = self.w
-        return 2.0 * self.T * self.scored_chunks() * w.hr * w.d
+        return 2.0 * self.timed_rows() * self.scored_chunks() * w.hr * w.d
 
     def check_planted(self):
         """Every layer's routed set must be its planted set (a property of the inputs)."""
@@ -562,6 +576,127 @@ class Routed:
                 if set(got[s].tolist()) != set(self.plans[l].docs[s]):
                     bad += 1
         return bad
+
+
+class Generate(Routed):
+    """Prefill, then generation: per sequence, every layer routes and attends the
+    prefill rows (causal over them), then each of `gen_steps` decoded tokens
+    goes through every layer: route its routing row against the whole bank,
+    gather, attend over the selected documents plus the local context so far
+    (prefill rows and the tokens generated before it, 129 .. 192 keys for the
+    1M workload). ["MSA: Memory Sparse Attention", Inference Pipeline: routing,
+    then generation over the assembled sparse context]"""
+
+    def __init__(self, w: synth.Workload, args, dev: int):
+        if not w.prefill_rows:
+            raise SystemExit(f"workload {w.name} has no prefill rows")
+        P, G = w.prefill_rows, args.gen_steps
+        w.route_rows = w.attn_rows = w.loc_len = P
+        super().__init__(w, args, dev)  # banks; the prefill step's rows, local keys, outputs, workspaces
+        import torch
+        msa, L, S, k, kk = self.msa, self.L, self.S, self.k, self.kk
+        hr, hkv, hq, d = w.hr, w.hkv, w.hq, w.d
+        self.P, self.G = P, G
+        stride = P + G  # local rows per sequence: the prefill rows, then one per generated token
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+        # one new planted routing row per sequence and step
+        self.qso_dec = np.arange(S + 1, dtype=np.int32)
+        qr_dec, self.plans_dec = [], []
+        for l in range(L):
+            def key_rows(c, l=l):
+                return synth.bits_to_f64(synth.normal_bf16_host(hr * d, synth.tid("kbar_r", l), index0=c * hr * d)
+                                         ).reshape(hr, d)
+            rows_l, plans_l = [], []
+            for t in range(G):
+                qr, _, plan = synth.make_routing_queries(key_rows, self.dco, [1] * S, k, w.n_needles, hr, d, l,
+                                                         call=1 + t)
+                rows_l.append(qr)
+                plans_l.append(plan)
+            qr_dec.append(np.stack(rows_l))
+            self.plans_dec.append(plans_l)
+        self.qr_dec = up(np.stack(qr_dec))  # [L, G, S, hr, d]
+        self.q_dec = up(synth.normal_bf16_host(L * G * S * hq * d, synth.tid("q_att", 7)).reshape(L, G, S, hq, d))
+        # local K/V: sequence s holds rows s * stride .. s * stride + P + G - 1 (prefill rows first)
+        kl = synth.normal_bf16_host(L * S * stride * hkv * d, synth.tid("k_loc", 7)).reshape(L, S * stride, hkv, d)
+        vl = synth.normal_bf16_host(L * S * stride * hkv * d, synth.tid("v_loc", 7)).reshape(L, S * stride, hkv, d)
+        self.kl_gen, self.vl_gen = up(kl), up(vl)
+        self.loc_off_gen = np.arange(S + 1, dtype=np.int32) * stride
+        self.ids_dec = torch.empty((L, G, S, kk), dtype=torch.int32, device="cuda")
+        self.sc_dec = torch.empty((L, G, S, kk), dtype=torch.float32, device="cuda")
+        self.out_dec = torch.empty((L, G, S, hq, d), dtype=torch.bfloat16, device="cuda")
+        # the attention workspace holds the prefill call's and the last decoding call's
+        need = max(msa.attend_workspace(*a, pos_offset=self.pos_offset, rope_theta=w.rope_theta)
+                   for a in (self._attend_args(0), self._dec_args(0, G - 1)))
+        self.ws_attend = torch.empty(need, dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def _attend_args(self, l):  # the prefill rows, causal over the first P local keys
+        if not hasattr(self, "kl_gen"):  # the base class sizing its workspace: replaced below
+            return super()._attend_args(l)
+        mk, mv = self.banks[l].kbar, self.banks[l].vbar
+        return (self.q_d[l], self.q_seq_off, np.zeros(self.S, np.int32), self.kl_gen[l], self.vl_gen[l],
+                self.loc_off_gen, mk, mv, self.sel_off, self.sel, self.cap)
+
+    def _dec_args(self, l, t):  # token t: active index P + t sees local keys 0 .. P + t
+        mk, mv = self.banks[l].kbar, self.banks[l].vbar
+        return (self.q_dec[l, t], self.qso_dec, np.full(self.S, self.P + t, np.int32), self.kl_gen[l], self.vl_gen[l],
+                self.loc_off_gen, mk, mv, self.sel_off, self.sel, self.cap)
+
+    def decode_layer(self, l, t, ev=None):
+        msa = self.msa
+        if ev is not None:
+            msa.score_events(ev[0], ev[1])
+        msa.route(self.banks[l], self.qr_dec[l, t], self.qso_dec, self.k, self.ids_dec[l, t], self.sc_dec[l, t],
+                  self.ws_route, eps=self.w.eps)
+        msa.gather(self.banks[l], self.ids_dec[l, t], self.k, self.sel_off, self.sel)
+        msa.attend(*self._dec_args(l, t), self.out_dec[l, t], self.ws_attend, pos_offset=self.pos_offset,
+                   rope_theta=self.w.rope_theta)
+
+    def prefill(self):
+        for l in range(self.L):
+            self.layer(l)
+
+    def step(self, evs=None):
+        self.prefill()
+        for t in range(self.G):
+            for l in range(self.L):  # the token passes through every layer
+                self.decode_layer(l, t, None if evs is None or t != self.G - 1 else evs[l])
+
+    def timed_rows(self) -> int:  # the roofline times the last token's decode scorer
+        return self.S
+
+    def units_per_step(self) -> float:
+        return float(self.w.memory_tokens) * self.S * self.L * (1 + self.G)
+
+    def check_planted(self):
+        bad = super().check_planted()
+        for l in range(self.L):
+            got = self.ids_dec[l].cpu().numpy()
+            for t in range(self.G):
+                for s in range(self.S):
+                    if set(got[t, s].tolist()) != set(self.plans_dec[l][t].docs[s]):
+                        bad += 1
+        return bad
+
+    def prefill_ms(self, reps: int = 5) -> float:
+        """Device time of the prefill part alone (a replayed CUDA graph of it)."""
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            self.prefill()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps
 
 
 class Encode:
@@ -639,6 +774,63 @@ def cpu_baseline(w: synth.Workload, max_chunks: int | None = None, layer: int = 
     total = t_route + t_att
     return dict(tokens=n_tok * S, seconds=total, route_s=t_route, attend_s=t_att, chunks=C, docs=dco.size - 1,
                 layer_chunks=int(w.index()[0][-1]), full_docs=D)
+
+
+def host_description() -> dict:
+    """The host cores the CPU baseline ran on."""
+    n = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": n, "cpu_model": model}
+
+
+def _cpu_all_cores_worker(name, over, max_chunks, layer, barrier, out):
+    w = synth.workload(name)
+    for k, v in over.items():
+        setattr(w, k, v)
+    barrier.wait(timeout=600)  # the data is generated; time the oracle with every process running
+    out.put(cpu_baseline(w, max_chunks=max_chunks, layer=layer))
+
+
+def cpu_baseline_all_cores(w: synth.Workload, max_chunks: int, max_procs: int = 16) -> dict:
+    """The same single-threaded oracle in P processes at once (one per core, up
+    to max_procs), each on a different layer's bounded sample: the host's
+    all-core throughput without threading the oracle. Processes are spawned
+    (not forked), so they never inherit a CUDA context."""
+    import multiprocessing as mpc
+    n = host_description()["nproc"]
+    P = max(1, min(n, max_procs))
+    over = {k: getattr(w, k) for k in ("n_seq", "route_rows", "attn_rows", "loc_len")}
+    ctx = mpc.get_context("spawn")
+    barrier, out = ctx.Barrier(P), ctx.Queue()
+    procs = [ctx.Process(target=_cpu_all_cores_worker, args=(w.name, over, max_chunks, i % w.n_layers, barrier, out))
+             for i in range(P)]
+    for p_ in procs:
+        p_.start()
+    import queue
+    res, t_end = [], time.monotonic() + 1800
+    try:
+        while len(res) < P:
+            try:
+                res.append(out.get(timeout=5))
+            except queue.Empty:
+                if any(p_.exitcode not in (None, 0) for p_ in procs) or time.monotonic() > t_end:
+                    raise RuntimeError("an all-core CPU baseline process failed or ran out of time")
+    finally:
+        for p_ in procs:
+            p_.join(timeout=60)
+            if p_.is_alive():
+                p_.kill()
+    tokens = sum(r["tokens"] for r in res)
+    slowest = max(r["seconds"] for r in res)
+    return {"value": tokens / slowest, "processes": P, "seconds": slowest, "chunks_per_process": res[0]["chunks"]}
 
 
 def encode_cpu_baseline(w: synth.Workload, n_docs: int = 2):
@@ -742,7 +934,12 @@ def run_ours(args):
             raise SystemExit(f"workload {w.name} has no prefill rows")
         w.route_rows = w.attn_rows = w.loc_len = w.prefill_rows
     metric, unit = metric_of(w.name)
-    eng = Encode(w, args, local) if w.name == "encode" else Routed(w, args, local)
+    if w.name == "encode":
+        eng = Encode(w, args, local)
+    elif args.mode == "generate":
+        eng = Generate(w, args, local)
+    else:
+        eng = Routed(w, args, local)
     L = eng.L
 
     def barrier():
@@ -764,6 +961,7 @@ def run_ours(args):
     if w.name != "encode" and args.mode != "interleave":
         bad = eng.check_planted()
         planted_ok = bad == 0
+        planted_sets = eng.L * eng.S * (1 + (eng.G if args.mode == "generate" else 0))
 
     # ---- timed region: K steps, inputs resident in HBM
     mp_ranks = getattr(eng, "mp_ranks", False)
@@ -821,13 +1019,13 @@ def run_ours(args):
 
     # ---- end to end through the public API: host inputs in, host results out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.mode != "generate":  # generate: the line reports the device-resident sequence
         e2e = run_e2e(eng, w, args, world, unit)
 
     peak, peak_kind = measured_peaks()
     # the library picks the many-row (tensor-bound) scorer above 64 query rows
     many_rows = w.name != "encode" and w.hr == 8 and (
-        args.score_kernel == "tc_rows" or (args.score_kernel == "auto" and eng.T > 64))
+        args.score_kernel == "tc_rows" or (args.score_kernel == "auto" and eng.timed_rows() > 64))
     if many_rows:
         kflops = eng.score_flops_per_launch()
         tpeak, tpeak_kind = measured_tensor_peak()
@@ -866,9 +1064,23 @@ def run_ours(args):
             cpu = {"value": r["tokens"] / r["seconds"], "unit": unit, "cores": 1, "kind": "oracle",
                    "sample": (f"one routing layer ({r['chunks']} chunks, {r['tokens']} memory tokens x sequences): "
                               f"route {r['route_s']:.1f} s + gather + attend {r['attend_s']:.2f} s, single thread")}
+        cpu["host"] = host_description()
+        if w.name != "encode" and not args.no_cpu_all_cores:
+            # a few seconds of work per process: fewer chunks when many query rows are scored
+            ac = cpu_baseline_all_cores(w, max_chunks=max(10_000, 200_000 // (w.n_seq * w.route_rows)))
+            cpu["all_cores"] = {"value": ac["value"], "unit": unit, "cores": ac["processes"], "kind": "oracle",
+                                "sample": (f"{ac['processes']} single-threaded oracle processes at once, each one "
+                                           f"layer's first {ac['chunks_per_process']} chunks (route + gather + "
+                                           f"attend), slowest {ac['seconds']:.1f} s")}
 
     extra = {"decode_latency_us_per_layer": 1e3 * ms / L, "cuda_graph": graph is not None, "mode": args.mode}
-    if w.name != "encode" and graph is not None and args.mode in ("decode", "train"):
+    if args.mode == "generate":
+        pf = eng.prefill_ms()
+        extra.update({"gen_steps": eng.G, "prefill_rows": eng.P, "prefill_ms": pf,
+                      "decode_us_per_token": 1e3 * (ms - pf) / eng.G,
+                      "decode_us_per_token_per_layer": 1e3 * (ms - pf) / eng.G / L,
+                      "local_keys": f"{eng.P + 1}..{eng.P + eng.G}"})
+    if w.name != "encode" and graph is not None and args.mode in ("decode", "train", "generate"):
         # the routing call as a whole (query norms, scoring, top-k), warm, inside a replayed graph
         st = eng.stage_times_graph()
         extra["stage_us_per_layer_graph"] = st
@@ -886,6 +1098,8 @@ def run_ours(args):
         extra["step"] = "prefill"
     if planted_ok is not None:
         extra["planted_sets_retrieved"] = planted_ok
+        if not planted_ok:  # the planted sets are a property of the inputs; the parity tests check the kernels
+            extra["planted_sets_missed"] = f"{bad} of {planted_sets}"
     if w.name != "encode" and w.content_on_host:
         extra["host_content_banks"] = eng.n_content
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
