@@ -23,11 +23,15 @@
 // When (tiles x kv heads) would not fill the GPU, the key blocks are split
 // across CTAs, each writing an unnormalised partial that the last one to
 // finish merges by log-sum-exp.
-// The rotated queries and local keys are fp32; each is split into a bf16 high
-// part and the bf16 rounding of the remainder, and S sums Qhi Khi + Qlo Khi +
-// Qhi Klo (the Qlo Klo term is below 2^-16 of the product), so the logits keep
-// fp32 accuracy. The pooled memory keys are bf16 already (exact). V is staged
-// transposed, so every operand is K-major with the 128-byte swizzle.
+// The rotated queries and local keys are split into a bf16 high part and the
+// bf16 rounding of the remainder (the local keys by rope_rows), and S sums
+// Qhi Khi + Qlo Khi + Qhi Klo (the Qlo Klo term is below 2^-16 of the
+// product), so the logits keep fp32 accuracy. The pooled memory keys are bf16
+// already (exact). Key blocks are staged two deep: the next block's key and
+// value rows are copied by cp.async (keys straight into their swizzled
+// places) while the current block's S, softmax and P.V run; the values are
+// then transposed shared-to-shared, so every MMA operand is K-major with the
+// 128-byte swizzle.
 // Every mbarrier wait is bounded in time, and every warp is reconverged
 // (__all_sync) after it: lanes leave a polling loop on different iterations,
 // and a diverged warp would run the softmax lane group by lane group.
@@ -46,16 +50,23 @@ constexpr int kNK = 64;           // keys per block
 constexpr int kThreadsTc = 256;  // 8 warps: (lane quadrant, half) pairs
 constexpr int kQAtom = kVec * 128;  // 16 KB: 128 rows x 64 dims (bf16)
 constexpr int kKAtom = kNK * 128;   // 8 KB: 64 keys x 64 dims
+constexpr int kVRow = 272;          // bytes per staged value row (256 + 16)
 constexpr int offQhi = 0;
 constexpr int offQlo = offQhi + 2 * kQAtom;
-constexpr int offKhi = offQlo + 2 * kQAtom;
-constexpr int offKlo = offKhi + 2 * kKAtom;
-constexpr int offVT = offKlo + 2 * kKAtom;  // 128 dims x 64 keys
-constexpr int offP = offVT + 128 * 128;     // 128 vectors x 64 keys
-constexpr int offIdx = offP + kVec * 128;  // 64 bank-row indices
-constexpr int offMax = offIdx + kNK * 8;   // [2][128] block maxima, then the two partial sums
+constexpr int offStage = offQlo + 2 * kQAtom;  // two stages of one key block each:
+constexpr int stKhi = 0;                       //   keys (bf16, or the high halves), 2 atoms
+constexpr int stKlo = stKhi + 2 * kKAtom;      //   low halves of local keys, 2 atoms
+constexpr int stV = stKlo + 2 * kKAtom;        //   value rows as stored [64][272 B]
+constexpr int kStageTc = stV + kNK * kVRow;    // 50,176 B
+constexpr int offVT = offStage + 2 * kStageTc;  // 128 dims x 64 keys
+constexpr int offP = offVT + 128 * 128;         // 128 vectors x 64 keys
+constexpr int offIdx = offP + kVec * 128;       // [2 blocks][64] bank-row indices
+constexpr int offMax = offIdx + 2 * kNK * 8;    // [2][128] block maxima, then the two partial sums
 constexpr int offBar = offMax + 2 * kVec * 4;
 constexpr int kSmemTc = 1024 + offBar + 64;
+static_assert(kStageTc % 1024 == 0 && offStage % 1024 == 0 && offVT % 1024 == 0 && offP % 1024 == 0,
+              "128-byte-swizzle atoms start on 1024-byte boundaries");
+static_assert(kSmemTc <= 227 * 1024, "shared memory per CTA");
 constexpr int kTmemCols = 256;  // S: columns 0..63, O block: 128..255
 // instruction descriptors: D fp32, A/B bf16, K-major; M = 128; N = 64 or 128
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNK >> 3) << 17) | (8u << 24);
@@ -63,6 +74,13 @@ constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(12
 
 // 16-byte piece c (0..7) of row r of a 128-byte-swizzled K-major atom.
 __device__ __forceinline__ uint8_t* swz(uint8_t* atom, int r, int c) { return atom + r * 128 + ((c ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ void cp16_tc(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit_tc() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait_tc() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float bf_round(float x) { return __uint_as_float(f2bf_bits(x) << 16); }
 
@@ -81,10 +99,10 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
 __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int64_t* s_idx = reinterpret_cast<int64_t*>(smem + offIdx);  // bank rows of this block's memory keys
+  int64_t* s_idx = reinterpret_cast<int64_t*>(smem + offIdx);  // [2][64] bank rows of two blocks' memory keys
   float* s_max = reinterpret_cast<float*>(smem + offMax);      // [half][vector]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + offBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + offBar);  // [0]: S committed, [1]: P.V committed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -105,7 +123,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   const int gv = vvalid ? g0 + rr : -1;
 
   if (tid == 0) {
-    mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(&bar[0]), 1);
+    mbar_init(smem_u32(&bar[1]), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -124,6 +143,53 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   const int64_t per = (n_blocks + p.n_splits - 1) / p.n_splits;
   const int64_t k_begin = min(n_keys, (int64_t)sp_idx * per * kNK);
   const int64_t k_end = min(n_keys, k_begin + per * kNK);
+  const int nblk = (int)((k_end - k_begin + kNK - 1) / kNK);
+
+  // Key blocks are staged two deep: block b + 1's rows are copied by cp.async
+  // while block b's S, softmax and P.V run. The bank row of memory key j of
+  // block b is read from the selection list one block before the copy.
+  auto load_idx = [&](int b, int j) -> int64_t {
+    const int64_t key = k_begin + (int64_t)b * kNK + j;
+    if (b >= nblk || key >= k_end || key >= n_mem) return -1;
+    return p.sel_chunk ? __ldcg(p.sel_chunk + mem_base + key) : mem_base + key;
+  };
+  auto issue = [&](int b) {
+    if (b < nblk) {
+      uint8_t* stg = smem + offStage + (b & 1) * kStageTc;
+      const int64_t kb = k_begin + (int64_t)b * kNK;
+      const int nb = (int)min((int64_t)kNK, k_end - kb);
+      const bool has_local = kb + nb > n_mem;
+      const int64_t* idx = s_idx + (b & 1) * kNK;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // 64 rows x 16 pieces of 16 bytes; 16 threads per row
+        const int id = tid + u * kThreadsTc;
+        const int jj = id >> 4, c = id & 15;
+        const int64_t key = kb + jj;
+        uint8_t* dk = swz(stg + stKhi + (c >> 3) * kKAtom, jj, c & 7);
+        uint8_t* dl = swz(stg + stKlo + (c >> 3) * kKAtom, jj, c & 7);
+        uint8_t* dv = stg + stV + jj * kVRow + 16 * c;
+        if (jj < nb && key < n_mem) {
+          const size_t off = ((size_t)idx[jj] * row_stride + (size_t)kvh * kHeadDim) * 2 + 16 * c;
+          cp16_tc(dk, reinterpret_cast<const uint8_t*>(p.mem_k) + off);
+          cp16_tc(dv, reinterpret_cast<const uint8_t*>(p.mem_v) + off);
+          if (has_local) *reinterpret_cast<uint4*>(dl) = make_uint4(0, 0, 0, 0);
+        } else if (jj < nb) {  // a local key: rotated by rope_rows, bf16 high halves then low halves
+          const size_t lrow = (size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh;
+          const uint8_t* kr = reinterpret_cast<const uint8_t*>(p.krot) + lrow * 512;
+          cp16_tc(dk, kr + 16 * c);
+          cp16_tc(dl, kr + 256 + 16 * c);
+          cp16_tc(dv, reinterpret_cast<const uint8_t*>(p.v_loc + lrow * kHeadDim) + 16 * c);
+        } else {
+          *reinterpret_cast<uint4*>(dv) = make_uint4(0, 0, 0, 0);  // P is 0 here; 0 x NaN would not be
+        }
+      }
+    }
+    cp_commit_tc();
+  };
+  if (tid < kNK) {
+    s_idx[tid] = load_idx(0, tid);
+    s_idx[kNK + tid] = load_idx(1, tid);
+  }
 
   {  // Q (high and low parts): this thread stages its vector's 64-dimension atom hs
     const float4* qv = reinterpret_cast<const float4*>(
@@ -159,115 +225,83 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   // of the O row in TMEM), so P <= 2^11.5 and P.V accumulates in TMEM across
   // blocks. l_own sums this thread's keys only; the halves add at the end.
   float m_ref = -INFINITY, l_own = 0.f;
-  uint32_t phase = 0;
-  bool ok = true, pv_pending = false;
-  int blk = 0;
+  uint32_t phase_s = 0, phase_pv = 0;
+  bool ok = true;
+  int pv_issued = 0;
 
-  for (int64_t kb = k_begin; kb < k_end; kb += kNK, ++blk) {
-    const int nb = (int)min((int64_t)kNK, k_end - kb);
-    const bool has_local = kb + nb > n_mem;
-    if (pv_pending) {  // the previous block's P.V still reads V^T and P
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
-      phase ^= 1;
-      pv_pending = false;
-      if (!__syncthreads_and(ok)) { ok = false; break; }
-      tc_fence_after();
+  // S of block b goes to TMEM columns 64 (b & 1) .. + 63 (O takes 128 .. 255),
+  // so block b + 1's S runs on the tensor cores while block b's softmax runs.
+  auto issue_s = [&](int b) {  // one thread; block b's rows are in its stage and visible to the async proxy
+    const int64_t kb = k_begin + (int64_t)b * kNK;
+    const bool has_local = kb + (int)min((int64_t)kNK, k_end - kb) > n_mem;
+    const uint8_t* stg = smem + offStage + (b & 1) * kStageTc;
+    const uint32_t ds = tmem + (uint32_t)(64 * (b & 1));
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t qa = (uint32_t)((k >> 2) * kQAtom + (k & 3) * 32);
+      const uint32_t ko = (uint32_t)((k >> 2) * kKAtom + (k & 3) * 32);
+      const uint64_t dkhi = sw128_desc(smem_u32(stg + stKhi) + ko);
+      tc_mma(ds, sw128_desc(smem_u32(smem + offQhi) + qa), dkhi, kIdescS, k > 0 ? 1u : 0u);
+      tc_mma(ds, sw128_desc(smem_u32(smem + offQlo) + qa), dkhi, kIdescS, 1u);
+      if (has_local)
+        tc_mma(ds, sw128_desc(smem_u32(smem + offQhi) + qa), sw128_desc(smem_u32(stg + stKlo) + ko), kIdescS, 1u);
     }
-    if (tid < nb && kb + tid < n_mem)
-      s_idx[tid] = p.sel_chunk ? __ldg(p.sel_chunk + mem_base + kb + tid) : mem_base + kb + tid;
+    tc_commit(smem_u32(&bar[0]));
+  };
+  issue(0);
+  issue(1);
+  if (nblk > 0) {
+    cp_wait_tc<1>();  // block 0's copies (this thread's)
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
+    if (tid == 0) issue_s(0);
+  }
 
-    {  // ---- K (high, low): 64 keys x 16 pieces of 8 dims, 4 pieces per thread
-      uint4 raw[4];
-      float4 fa[4], fb[4];
-      int kind[4];  // 0 none, 1 memory, 2 local
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = tid + u * kThreadsTc;
-        const int jj = idx >> 4, c = idx & 15;
-        const int64_t key = kb + jj;
-        kind[u] = jj >= nb ? 0 : key < n_mem ? 1 : 2;
-        raw[u] = make_uint4(0, 0, 0, 0);
-        fa[u] = fb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (kind[u] == 1) {
-          raw[u] = __ldg(reinterpret_cast<const uint4*>(p.mem_k + (size_t)s_idx[jj] * row_stride +
-                                                        (size_t)kvh * kHeadDim + 8 * c));
-        } else if (kind[u] == 2) {
-          const float4* kr = reinterpret_cast<const float4*>(
-              p.krot + ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim);
-          fa[u] = __ldg(kr + 2 * c);
-          fb[u] = __ldg(kr + 2 * c + 1);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = tid + u * kThreadsTc;
-        const int jj = idx >> 4, c = idx & 15;
-        uint4 hi = raw[u], lo = make_uint4(0, 0, 0, 0);
-        if (kind[u] == 2) {
-          const float f[8] = {fa[u].x, fa[u].y, fa[u].z, fa[u].w, fb[u].x, fb[u].y, fb[u].z, fb[u].w};
-          split8(f, hi, lo);
-        }
-        *reinterpret_cast<uint4*>(swz(smem + offKhi + (c >> 3) * kKAtom, jj, c & 7)) = hi;
-        if (has_local) *reinterpret_cast<uint4*>(swz(smem + offKlo + (c >> 3) * kKAtom, jj, c & 7)) = lo;
-      }
+  for (int b = 0; b < nblk; ++b) {
+    const int64_t kb = k_begin + (int64_t)b * kNK;
+    const int nb = (int)min((int64_t)kNK, k_end - kb);
+    uint8_t* stg = smem + offStage + (b & 1) * kStageTc;
+    const int64_t r2 = tid < kNK ? load_idx(b + 2, tid) : -1;  // stored before block b + 2's copies go out
+    // ---- S of block b is done; so is block b - 1's P.V (V^T, P and O are free)
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar[0]), phase_s, abort_flag));
+    phase_s ^= 1;
+    if (ok && b > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar[1]), phase_pv, abort_flag));
+      phase_pv ^= 1;
     }
-    {  // V^T: this thread takes keys 2 jp, 2 jp + 1 and dimensions 16 dg .. 16 dg + 15
+    cp_wait_tc<0>();  // this thread's copies of block b + 1
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc_fence_after();
+    if (tid == 0 && b + 1 < nblk) issue_s(b + 1);  // overlaps this block's softmax
+
+    {  // V^T from the staged rows: this thread takes keys 2 jp, 2 jp + 1 and dimensions 16 dg .. 16 dg + 15
       const int jp = tid & 31, dg = tid >> 5;
       uint4 x[2][2];
 #pragma unroll
-      for (int k2 = 0; k2 < 2; ++k2) {
-        const int jj = 2 * jp + k2;
-        const int64_t key = kb + jj;
-        const uint16_t* vr = nullptr;
-        if (jj < nb && key < n_mem)
-          vr = p.mem_v + (size_t)s_idx[jj] * row_stride + (size_t)kvh * kHeadDim;
-        else if (jj < nb)
-          vr = p.v_loc + ((size_t)(p.loc_off[s] + (key - n_mem)) * p.hkv + kvh) * kHeadDim;
+      for (int k2 = 0; k2 < 2; ++k2)
 #pragma unroll
         for (int i = 0; i < 2; ++i)
-          x[k2][i] = vr ? __ldg(reinterpret_cast<const uint4*>(vr + 16 * dg) + i) : make_uint4(0, 0, 0, 0);
-      }
+          x[k2][i] = *reinterpret_cast<const uint4*>(stg + stV + (2 * jp + k2) * kVRow + 32 * dg + 16 * i);
 #pragma unroll
       for (int d = 0; d < 16; ++d) {
         const uint4& a = x[0][d >> 3];
-        const uint4& b = x[1][d >> 3];
+        const uint4& bq = x[1][d >> 3];
         const int w = (d >> 1) & 3;
         const uint32_t wa = w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
-        const uint32_t wb = w == 0 ? b.x : w == 1 ? b.y : w == 2 ? b.z : b.w;
+        const uint32_t wb = w == 0 ? bq.x : w == 1 ? bq.y : w == 2 ? bq.z : bq.w;
         const int dim = 16 * dg + d;
         *reinterpret_cast<uint32_t*>(swz(smem + offVT, dim, jp >> 2) + 4 * (jp & 3)) =
             __byte_perm(wa, wb, (d & 1) ? 0x7632 : 0x5410);
       }
     }
-    fence_proxy_async_smem();  // the MMAs read these bytes through the async proxy
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- S = Q K^T
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t qa = (uint32_t)((k >> 2) * kQAtom + (k & 3) * 32);
-        const uint32_t ko = (uint32_t)((k >> 2) * kKAtom + (k & 3) * 32);
-        const uint64_t dkhi = sw128_desc(smem_u32(smem + offKhi) + ko);
-        tc_mma(tmem, sw128_desc(smem_u32(smem + offQhi) + qa), dkhi, kIdescS, k > 0 ? 1u : 0u);
-        tc_mma(tmem, sw128_desc(smem_u32(smem + offQlo) + qa), dkhi, kIdescS, 1u);
-        if (has_local)
-          tc_mma(tmem, sw128_desc(smem_u32(smem + offQhi) + qa), sw128_desc(smem_u32(smem + offKlo) + ko), kIdescS,
-                 1u);
-      }
-      tc_commit(smem_u32(bar));
-    }
-    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
-    phase ^= 1;
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    tc_fence_after();
 
     // ---- softmax: this thread's 32 keys (32 hs .. 32 hs + 31) of its vector
     float sv[32];
-    tmem_ld32(tmem + lane_base + 32 * hs, sv);
+    tmem_ld32(tmem + (uint32_t)(64 * (b & 1)) + lane_base + 32 * hs, sv);
     tmem_ld_wait();
     // Logits in log2 units (scale * log2 e) so that P = 2^(s - m_ref). Key j
     // of the block is visible to this vector iff j < jvis: the block's memory
@@ -283,7 +317,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
       bmo = fmaxf(bmo, sv[j]);
     }
     s_max[hs * kVec + v] = bmo;
-    __syncthreads();
+    if (tid < kNK) s_idx[(b & 1) * kNK + tid] = r2;  // block b + 2's rows (block b's copies went out long ago)
+    __syncthreads();  // also: every thread has read block b's staged values
+    issue(b + 2);     // into block b's stage (its S is done, its values transposed)
     const float bm = fmaxf(s_max[v], s_max[kVec + v]);
     const bool move = bm > m_ref + 11.5f;  // 2^11.5 ~ e^8; also when m_ref is -inf and bm finite
     const float corr = !move ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - bm));
@@ -303,7 +339,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
     }
     l_own = l_own * corr + sum;
     // rescale this thread's half of the O row when any lane of the warp moved its reference
-    if (blk > 0 && __any_sync(0xffffffffu, move)) {
+    if (b > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float t[16];
@@ -319,27 +355,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
     tc_fence_before();
     __syncthreads();
 
-    // ---- O += P V (accumulated in TMEM; waited for before V^T and P are reused)
+    // ---- O += P V (accumulated in TMEM; waited for before V^T, P and O are touched again)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < kNK / 16; ++k)
         tc_mma(tmem_o, sw128_desc(smem_u32(smem + offP) + k * 32), sw128_desc(smem_u32(smem + offVT) + k * 32),
-               kIdescO, (blk > 0 || k > 0) ? 1u : 0u);
-      tc_commit(smem_u32(bar));
+               kIdescO, (b > 0 || k > 0) ? 1u : 0u);
+      tc_commit(smem_u32(&bar[1]));
     }
-    pv_pending = true;
+    ++pv_issued;
   }
-  if (ok && pv_pending) {
-    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), phase, abort_flag));
-    phase ^= 1;
+  if (ok && pv_issued > 0) {  // the last block's P.V
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar[1]), phase_pv, abort_flag));
+    phase_pv ^= 1;
     ok = __syncthreads_and(ok);
   }
   if (!ok && tid == 0) {  // a wait ran out: let the MMAs in flight finish (bounded) before TMEM is freed
     const uint64_t t0 = globaltimer();
-    while (!mbar_try(smem_u32(bar), phase ^ 1) && globaltimer() - t0 < kWaitLimitNs) {
+    while ((!mbar_try(smem_u32(&bar[0]), phase_s ^ 1) || !mbar_try(smem_u32(&bar[1]), phase_pv ^ 1)) &&
+           globaltimer() - t0 < kWaitLimitNs) {
     }
   }
+  cp_wait_tc<0>();  // no copy in flight
+  const int blk = ok ? nblk : 0;
   tc_fence_after();
   // the vector's sum over both halves
   s_max[hs * kVec + v] = l_own;
