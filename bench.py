@@ -44,11 +44,18 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=["100m", "10m", "1m", "tiny", "encode"], default="100m")
     p.add_argument("--score-kernel", choices=["auto", "simt", "tc", "tc_rows"], default="auto")
-    p.add_argument("--attend-kernel", choices=["auto", "split", "tc", "tc_dec"], default="auto")
+    p.add_argument("--attend-kernel", choices=["auto", "split", "tc", "tc_dec", "dec"], default="auto")
     p.add_argument("--attend-splits", type=int, default=0,
                    help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
+    p.add_argument("--dec-rot-keys", type=int, default=-1,
+                   help="decoding attention: largest per-CTA share of local keys it rotates itself "
+                        "(-1: the library's default; 0: always the separate rotation kernel)")
+    p.add_argument("--listing", choices=["routed", "gather"], default="routed",
+                   help="device-resident content: msa_attend lists the selected documents' chunks itself from "
+                        "the route's ids (routed, the default), or msa_gather lists them first (gather); content "
+                        "in host memory and --mode train always use msa_gather")
     p.add_argument("--content-layers", type=int, default=0,
                    help="host-tier content banks to allocate; layer l uses bank l mod this (0, the default: one "
                         "per layer if host RAM allows, else one shared by all layers)")
@@ -371,8 +378,11 @@ class Routed:
         self.out_all = torch.empty((self.L, self.Tq, w.hq, d), dtype=torch.bfloat16, device="cuda")
         self.out = [self.out_all[l] for l in range(self.L)]
         self.pos_offset = float(k)
+        # device-resident content: attend takes the route's ids (the routed form, no msa_gather)
+        self.routed = args.listing == "routed" and not self.on_host and args.mode != "train"
         a0 = self._attend_args(0)
-        self.ws_attend = torch.empty(msa.attend_workspace(*a0, pos_offset=self.pos_offset, rope_theta=w.rope_theta),
+        self.ws_attend = torch.empty(msa.attend_workspace(*a0, pos_offset=self.pos_offset, rope_theta=w.rope_theta,
+                                                          routed=self._routed(0, self.ids[0])),
                                      dtype=torch.uint8, device="cuda")
         self.mode = msa.GATHER_DEVICE_PULL if args.gather == "pull" else msa.GATHER_COPY_ENGINE
         self.run_mode = args.mode
@@ -430,13 +440,23 @@ class Routed:
             avail = 0
         return self.L if need < 0.6 * avail else 1
 
+    def _routed(self, l, ids):
+        """The routed-form argument of msa.attend for layer l's ids, or None."""
+        return (ids, self.banks[l].doc_chunk_off) if getattr(self, "routed", False) else None
+
+    def _listing(self):
+        """sel_off, sel_chunk of msa.attend: None for the routed form."""
+        if getattr(self, "routed", False):
+            return None, None
+        return self.sel_off, (None if self.on_host else self.sel)
+
     def _attend_args(self, l):
         if self.on_host:
-            mk, mv, sel = self.stage_k, self.stage_v, None
+            mk, mv = self.stage_k, self.stage_v
         else:
-            mk, mv, sel = self.banks[l].kbar, self.banks[l].vbar, self.sel
+            mk, mv = self.banks[l].kbar, self.banks[l].vbar
         return (self.q_d[l], self.q_seq_off, self.q_start, self.kl_d[l], self.vl_d[l], self.loc_off, mk, mv,
-                self.sel_off, sel, self.cap)
+                *self._listing(), self.cap)
 
     def layer(self, l, ev=None):
         msa = self.msa
@@ -476,11 +496,11 @@ class Routed:
             msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel, self.stage_k, self.stage_v,
                        mode=self.mode, doc_chunk_off_host=self.dco, top_ids_host=self.ids_host,
                        copy_stream=self.copy_stream, done_event=self.copy_done)
-        else:
+        elif not self.routed:
             msa.gather(self.banks[l], self.ids[l], self.k, self.sel_off, self.sel)
         if self.run_mode != "train":
             msa.attend(*self._attend_args(l), self.out[l], self.ws_attend, pos_offset=self.pos_offset,
-                       rope_theta=self.w.rope_theta)
+                       rope_theta=self.w.rope_theta, routed=self._routed(l, self.ids[l]))
             return
         a = self._attend_args(l)
         msa.attend(*a, self.out[l], self.ws_attend, out_f32=self.out_f32[l], lse=self.lse[l],
@@ -628,8 +648,9 @@ class Generate(Routed):
         self.sc_dec = torch.empty((L, G, S, kk), dtype=torch.float32, device="cuda")
         self.out_dec = torch.empty((L, G, S, hq, d), dtype=torch.bfloat16, device="cuda")
         # the attention workspace holds the prefill call's and the last decoding call's
-        need = max(msa.attend_workspace(*a, pos_offset=self.pos_offset, rope_theta=w.rope_theta)
-                   for a in (self._attend_args(0), self._dec_args(0, G - 1)))
+        need = max(msa.attend_workspace(*a, pos_offset=self.pos_offset, rope_theta=w.rope_theta,
+                                        routed=self._routed(0, ids))
+                   for a, ids in ((self._attend_args(0), self.ids[0]), (self._dec_args(0, G - 1), self.ids_dec[0, 0])))
         self.ws_attend = torch.empty(need, dtype=torch.uint8, device="cuda")
         torch.cuda.synchronize()
 
@@ -638,12 +659,12 @@ class Generate(Routed):
             return super()._attend_args(l)
         mk, mv = self.banks[l].kbar, self.banks[l].vbar
         return (self.q_d[l], self.q_seq_off, np.zeros(self.S, np.int32), self.kl_gen[l], self.vl_gen[l],
-                self.loc_off_gen, mk, mv, self.sel_off, self.sel, self.cap)
+                self.loc_off_gen, mk, mv, *self._listing(), self.cap)
 
     def _dec_args(self, l, t):  # token t: active index P + t sees local keys 0 .. P + t
         mk, mv = self.banks[l].kbar, self.banks[l].vbar
         return (self.q_dec[l, t], self.qso_dec, np.full(self.S, self.P + t, np.int32), self.kl_gen[l], self.vl_gen[l],
-                self.loc_off_gen, mk, mv, self.sel_off, self.sel, self.cap)
+                self.loc_off_gen, mk, mv, *self._listing(), self.cap)
 
     def decode_layer(self, l, t, ev=None):
         msa = self.msa
@@ -651,9 +672,10 @@ class Generate(Routed):
             msa.score_events(ev[0], ev[1])
         msa.route(self.banks[l], self.qr_dec[l, t], self.qso_dec, self.k, self.ids_dec[l, t], self.sc_dec[l, t],
                   self.ws_route, eps=self.w.eps)
-        msa.gather(self.banks[l], self.ids_dec[l, t], self.k, self.sel_off, self.sel)
+        if not self.routed:
+            msa.gather(self.banks[l], self.ids_dec[l, t], self.k, self.sel_off, self.sel)
         msa.attend(*self._dec_args(l, t), self.out_dec[l, t], self.ws_attend, pos_offset=self.pos_offset,
-                   rope_theta=self.w.rope_theta)
+                   rope_theta=self.w.rope_theta, routed=self._routed(l, self.ids_dec[l, t]))
 
     def prefill(self):
         for l in range(self.L):
@@ -860,10 +882,13 @@ def config_of(w, eng, args, extra=None):
         cfg.update({"chunks_per_layer": eng.C, "sequences": w.n_seq, "routing_rows_per_seq": w.route_rows,
                     "top_k": w.top_k, "hq": w.hq, "hkv": w.hkv, "local_tokens": w.loc_len,
                     "content": "pinned_host" if w.content_on_host else "hbm",
-                    "gather": args.gather if w.content_on_host else "hbm_index",
+                    "gather": args.gather if w.content_on_host else (
+                        "in_attend" if getattr(eng, "routed", False) else "hbm_index"),
                     "score_kernel": args.score_kernel, "attend_kernel": args.attend_kernel})
         if args.attend_splits:
             cfg["attend_splits"] = args.attend_splits
+        if args.dec_rot_keys >= 0:
+            cfg["dec_rot_keys"] = args.dec_rot_keys
     else:
         cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
     cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
@@ -926,6 +951,8 @@ def run_ours(args):
     msa.set_score_kernel(args.score_kernel)
     msa.set_attend_kernel(args.attend_kernel)
     msa.set_attend_splits(args.attend_splits)
+    if args.dec_rot_keys >= 0:
+        msa.set_dec_rot_keys(args.dec_rot_keys)
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs

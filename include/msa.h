@@ -304,6 +304,17 @@ msa_status msa_gather(const msa_gather_args* args, void* stream);
  *   out[r, h] = softmax(scale * q' . keys) @ values, lse[r, h] = log-sum-exp.
  * Memory row m of s is mem_k[sel_chunk[sel_off[s] + m]] (or, if sel_chunk is
  * NULL, mem_k[sel_off[s] + m], e.g. the staging buffer of msa_gather).
+ * Routed form (sel_off = sel_chunk = NULL, top_ids set): the call lists the
+ * memory rows itself, exactly as msa_gather would for device-resident content.
+ * The memory rows of s are the chunks of documents top_ids[s * top_k + j],
+ * j = 0 .. top_k - 1 in that order, each from doc_chunk_off[id] to
+ * doc_chunk_off[id + 1] - 1 (rows of mem_k/mem_v: a bank's kbar/vbar in device
+ * memory). top_ids is msa_route's output and doc_chunk_off the bank's, both on
+ * the device. An id outside [0, n_docs) lists nothing. max_sel must be at
+ * least every sequence's memory row count (top_k x the bank's max_doc_chunks
+ * always is); with less, the call stays inside its buffers but its result is
+ * unspecified. This form saves the msa_gather launch on the path route ->
+ * attend; msa_attend_backward does not take it (MSA_ERR_UNSUPPORTED).
  * out is bf16 (nearest even of the fp32 result); out_f32 and lse are optional.
  * max_sel >= sel_off[s+1] - sel_off[s] for every s sizes the split-K grid.
  * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16, n_seq <= 256. q, k_loc,
@@ -311,9 +322,11 @@ msa_status msa_gather(const msa_gather_args* args, void* stream);
  * workspace 256-byte aligned (MSA_ERR_INVALID_ARG / MSA_ERR_WORKSPACE).
  * How it runs (not part of the contract): when a sequence's query vectors
  * (rows x hq / hkv) fill at least 64, the logits and P.V run on the tensor
- * cores (the logits at fp32 accuracy, P rounded to bf16); otherwise a
- * decoding kernel on CUDA cores streams the key rows by cp.async, with
- * memory and local keys in separate CTAs merged by log-sum-exp.
+ * cores (the logits at fp32 accuracy, P rounded to bf16) after a kernel that
+ * rotates the queries and local keys; otherwise one decoding kernel rotates
+ * its own rows, streams the key rows by cp.async and runs the logits and P.V
+ * as warp-level MMAs, its key splits merged by log-sum-exp inside a
+ * thread-block cluster.
  * ---------------------------------------------------------------------- */
 typedef struct msa_attend_args {
   const uint16_t* q;          /* device [n_q, hq, d] bf16, not rotated */
@@ -326,7 +339,7 @@ typedef struct msa_attend_args {
   const int32_t* loc_off;     /* HOST [n_seq + 1] */
   const uint16_t* mem_k;      /* device (or mapped pinned host) [*, hkv, d] bf16 */
   const uint16_t* mem_v;
-  const int64_t* sel_off;     /* device [n_seq + 1] */
+  const int64_t* sel_off;     /* device [n_seq + 1], or NULL for the routed form */
   const int64_t* sel_chunk;   /* device [*] or NULL */
   int64_t max_sel;
   float pos_offset;           /* global RoPE offset of the active context (the pages: k) */
@@ -335,6 +348,12 @@ typedef struct msa_attend_args {
   uint16_t* out;              /* device out [n_q, hq, d] bf16 */
   float* out_f32;             /* device out [n_q, hq, d] or NULL */
   float* lse;                 /* device out [n_q, hq] or NULL */
+  /* routed form (used when top_ids != NULL; sel_off and sel_chunk must be NULL) */
+  const int32_t* top_ids;     /* device [n_seq, top_k]: msa_route's top_ids */
+  const int64_t* doc_chunk_off; /* device [n_docs + 1]: the bank's */
+  int64_t n_docs;
+  int32_t top_k;              /* 1 .. 4096 */
+  int32_t reserved2;
 } msa_attend_args;
 
 msa_status msa_attend_workspace(const msa_attend_args* args, size_t* bytes);

@@ -66,7 +66,8 @@ class AttendArgsC(ctypes.Structure):
                 ("hkv", i32), ("d", i32), ("reserved", i32), ("k_loc", P), ("v_loc", P), ("loc_off", P),
                 ("mem_k", P), ("mem_v", P), ("sel_off", P), ("sel_chunk", P), ("max_sel", i64),
                 ("pos_offset", f32), ("rope_theta", f32), ("scale", f32), ("out", P), ("out_f32", P),
-                ("lse", P)]
+                ("lse", P), ("top_ids", P), ("doc_chunk_off", P), ("n_docs", i64), ("top_k", i32),
+                ("reserved2", i32)]
 
 
 def _sig(name, args, res=ctypes.c_int):
@@ -85,6 +86,7 @@ _sig("msa_debug_set_pf_pair", [ctypes.c_int])
 _sig("msa_debug_wait_probe", [ctypes.c_void_p])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_set_attend_splits", [ctypes.c_int])
+_sig("msa_debug_set_dec_rot_keys", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
 _sig("msa_debug_score_events", [P, P], None)
@@ -167,6 +169,13 @@ def set_attend_splits(n: int) -> int:
     the previous setting. Workspace sizes follow it: query attend_workspace
     after changing it. Benchmarking control."""
     return int(_lib.msa_debug_set_attend_splits(int(n)))
+
+
+def set_dec_rot_keys(n: int) -> int:
+    """Largest per-CTA share of local keys the decoding attention kernel rotates
+    itself (0..256; 0: a separate rotation kernel always does); returns the
+    previous setting. Workspace sizes follow it. Testing control."""
+    return int(_lib.msa_debug_set_dec_rot_keys(int(n)))
 
 
 def wait_probe() -> None:
@@ -317,19 +326,24 @@ def gather(bank: BankLayer, top_ids, top_k: int, sel_off, sel_chunk, stage_k=Non
 # ------------------------------------------------------------------ attend
 
 def _attend_args(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
-                 max_sel, pos_offset, rope_theta, scale, out, out_f32, lse):
+                 max_sel, pos_offset, rope_theta, scale, out, out_f32, lse, routed=None):
+    """routed = (top_ids [n_seq, top_k] int32, doc_chunk_off [n_docs + 1] int64), both on the
+    device, for the routed form (sel_off and sel_chunk None)."""
     qso, qst, lo = _host_i32(q_seq_off), _host_i32(q_start), _host_i32(loc_off)
+    top_ids, dco = routed if routed is not None else (None, None)
     a = AttendArgsC(_ptr(q), qso.ctypes.data, qst.ctypes.data, qso.size - 1, q.shape[0], q.shape[1],
                     (k_loc if k_loc is not None else mem_k).shape[1], q.shape[2], 0, _ptr(k_loc), _ptr(v_loc),
                     lo.ctypes.data, _ptr(mem_k), _ptr(mem_v), _ptr(sel_off), _ptr(sel_chunk), int(max_sel),
-                    float(pos_offset), float(rope_theta), float(scale), _ptr(out), _ptr(out_f32), _ptr(lse))
+                    float(pos_offset), float(rope_theta), float(scale), _ptr(out), _ptr(out_f32), _ptr(lse),
+                    _ptr(top_ids), _ptr(dco), dco.numel() - 1 if dco is not None else 0,
+                    top_ids.shape[1] if top_ids is not None else 0, 0)
     return a, (qso, qst, lo)
 
 
 def attend_workspace(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
-                     max_sel, pos_offset=16.0, rope_theta=1e6, scale=0.0) -> int:
+                     max_sel, pos_offset=16.0, rope_theta=1e6, scale=0.0, routed=None) -> int:
     a, keep = _attend_args(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
-                           max_sel, pos_offset, rope_theta, scale, q, None, None)
+                           max_sel, pos_offset, rope_theta, scale, q, None, None, routed)
     n = ctypes.c_size_t()
     _check(_lib.msa_attend_workspace(ctypes.byref(a), ctypes.byref(n)), "msa_attend_workspace")
     return n.value
@@ -337,9 +351,11 @@ def attend_workspace(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v,
 
 def attend(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk, max_sel,
            out, workspace, out_f32=None, lse=None, pos_offset=16.0, rope_theta=1e6, scale=0.0,
-           stream=None) -> None:
+           stream=None, routed=None) -> None:
+    """With routed = (top_ids, doc_chunk_off) and sel_off = sel_chunk = None, the call lists
+    the selected documents' chunks itself (the routed form of msa_attend)."""
     a, keep = _attend_args(q, q_seq_off, q_start, k_loc, v_loc, loc_off, mem_k, mem_v, sel_off, sel_chunk,
-                           max_sel, pos_offset, rope_theta, scale, out, out_f32, lse)
+                           max_sel, pos_offset, rope_theta, scale, out, out_f32, lse, routed)
     _check(_lib.msa_attend(ctypes.byref(a), _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream)), "msa_attend")
 

@@ -9,8 +9,8 @@
 //
 // Two kernels:
 //  1. rope_rows: rotates the query rows and the local keys once per call into
-//     fp32 copies (local keys as bf16 high + low halves for the decoding kernel
-//     of attend_dec.cu), and clears the merge tickets. Each angle is formed and
+//     fp32 copies (local keys as bf16 high + low halves for the tensor-core
+//     kernel of attend_tc.cu), and clears the merge tickets. Each angle is formed and
 //     reduced modulo 2*pi in double, so positions of any size keep full
 //     accuracy, and then evaluated with sincosf.
 //  2. attend_split: split-K flash decoding. A CTA owns one kv head, a tile of
@@ -56,21 +56,13 @@ struct Smem {
 // together).
 constexpr int kRopeHeads = 4;
 
-// An angle (radians, double) reduced to [-pi, pi] in double, as a float: sincosf
-// then evaluates it on its short, accurate range for positions of any size.
-__device__ __forceinline__ float reduced_angle(double ang) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  return (float)(ang - two_pi * rint(ang * inv_two_pi));
-}
-
 __global__ void rope_rows_kernel(const __grid_constant__ AttnParams p) {
   pdl_wait();
   pdl_trigger();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx < (int64_t)p.n_tiles * p.hkv) p.tickets[idx] = 0u;
+  if (p.tickets && idx < (int64_t)p.n_tiles * p.hkv) p.tickets[idx] = 0u;
   const int gq = (p.hq + kRopeHeads - 1) / kRopeHeads, gk = (p.hkv + kRopeHeads - 1) / kRopeHeads;
-  const int64_t nq = (int64_t)p.n_q * gq * 64;
+  const int64_t nq = p.rope_q ? (int64_t)p.n_q * gq * 64 : 0;
   const int64_t nk = (int64_t)p.n_loc * gk * 64;
   if (idx >= nq + nk) return;
   const bool is_q = idx < nq;
@@ -719,18 +711,21 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_dkdv_kernel(const __grid_
 
 struct Shape {
   int vec, rt, n_tiles, n_splits, n_loc;
-  bool tc;   // tensor-core kernel (many rows per sequence)
-  bool dec;  // decoding kernel (attend_dec.cu)
+  bool rot;   // decoding kernel: it rotates its own local keys (rope_rows does otherwise)
+  bool tc;    // tensor-core kernel (many rows per sequence)
+  bool dec;   // decoding kernel (attend_dec.cu)
+  bool list;  // routed form listed into the workspace first (every kernel but the decoding one)
 };
 
 // 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores, 4 decoding
 // kernel on CUDA cores (testing control)
 int g_attend_kernel = 0;
 int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
+int g_dec_rot_keys = 48;  // decoding kernel: largest local-key share per CTA it rotates itself
 
 // allow_tc: the forward may take the tensor-core kernel when the query
 // vectors of a sequence fill at least half of its 128-vector tile.
-Shape plan(const msa_attend_args& a, bool allow_tc) {
+Shape plan_kernel(const msa_attend_args& a, bool allow_tc) {
   Shape sh{};
   const int group = a.hq / a.hkv;
   int max_rows = 1;
@@ -780,9 +775,10 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
   }
   sh.n_loc = a.loc_off[a.n_seq];
   if (sh.dec) {
-    // one CTA per SM (the kernel takes ~165 KB of shared memory): key splits
+    // one CTA per SM (the kernel takes ~218 KB of shared memory): key splits
     // per (tile, kv head) while the grid is under 148 CTAs, each split an even
-    // share of the sequence's memory keys and of its local keys
+    // share of the sequence's memory keys and of its local keys; the splits of
+    // a (tile, kv head) are one cluster, so at most 8
     int max_lvis = 0;
     for (int s = 0; s < a.n_seq; ++s) {
       const int rows = a.q_seq_off[s + 1] - a.q_seq_off[s];
@@ -792,8 +788,12 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
     const int64_t pairs = std::max<int64_t>((int64_t)sh.n_tiles * a.hkv, 1);
     int64_t splits = g_attend_splits > 0 ? g_attend_splits : 148 / pairs;
     const int64_t cap = (a.max_sel + max_lvis + 63) / 64;  // at least one 64-key block each
-    splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, cap), 64));
+    splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, cap), kDecMaxSplits));
     sh.n_splits = (int)splits;
+    // a CTA rotates its own share of the local keys when that is at most
+    // g_dec_rot_keys: below that the work costs less than a kernel boundary
+    const int share = (int)((max_lvis + splits - 1) / splits);
+    sh.rot = share <= std::min(g_dec_rot_keys, kDecRotKeysMax);
     return sh;
   }
   const int64_t max_keys = a.max_sel + max_loc;
@@ -808,19 +808,40 @@ Shape plan(const msa_attend_args& a, bool allow_tc) {
   return sh;
 }
 
+Shape plan(const msa_attend_args& a, bool allow_tc) {
+  Shape sh = plan_kernel(a, allow_tc);
+  sh.list = a.sel_off == nullptr && !(sh.dec && a.top_k <= kDecRoutedMaxK);
+  return sh;
+}
+
 struct Layout {
-  size_t qrot, krot, part_o, part_ml, tickets, total;
+  size_t qrot, krot, part_o, part_ml, tickets, list_off, list_chunk, total;
 };
 
 Layout layout(const msa_attend_args& a, const Shape& sh) {
-  Layout L;
-  L.qrot = 0;
-  L.krot = L.qrot + align_up((size_t)a.n_q * a.hq * kHeadDim * 4, 256);
-  L.part_o = L.krot + align_up((size_t)(sh.n_loc > 0 ? sh.n_loc : 1) * a.hkv * kHeadDim * 4, 256);
-  const size_t np = sh.n_splits > 1 ? (size_t)a.n_q * a.hq * sh.n_splits : 0;
-  L.part_ml = L.part_o + align_up(np * kHeadDim * 4, 256);
-  L.tickets = L.part_ml + align_up(np * 8, 256);
-  L.total = L.tickets + align_up((size_t)sh.n_tiles * a.hkv * 4 + 4, 256);
+  Layout L{};
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = at;
+    at += align_up(bytes, 256);
+    return o;
+  };
+  if (sh.dec) {
+    // the decoding kernel: the local keys rotated by rope_rows (bf16 high and low halves, 512 B)
+    if (!sh.rot) L.krot = take((size_t)std::max(sh.n_loc, 1) * a.hkv * 2 * kHeadDim * 2);
+  } else {
+    L.qrot = take((size_t)a.n_q * a.hq * kHeadDim * 4);
+    L.krot = take((size_t)(sh.n_loc > 0 ? sh.n_loc : 1) * a.hkv * kHeadDim * 4);
+    const size_t np = sh.n_splits > 1 ? (size_t)a.n_q * a.hq * sh.n_splits : 0;
+    L.part_o = take(np * kHeadDim * 4);
+    L.part_ml = take(np * 8);
+    L.tickets = take((size_t)sh.n_tiles * a.hkv * 4 + 4);
+  }
+  if (sh.list) {  // the routed form's listing: n_seq x max_sel rows at most
+    L.list_off = take((size_t)(a.n_seq + 1) * 8);
+    L.list_chunk = take((size_t)std::max<int64_t>((int64_t)a.n_seq * a.max_sel, 1) * 8);
+  }
+  L.total = std::max<size_t>(at, 256);
   return L;
 }
 
@@ -847,15 +868,23 @@ namespace {
 void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, char* w, AttnParams& P) {
   P.q = a.q; P.k_loc = a.k_loc; P.v_loc = a.v_loc; P.mem_k = a.mem_k; P.mem_v = a.mem_v;
   P.sel_off = a.sel_off; P.sel_chunk = a.sel_chunk;
+  P.top_ids = a.top_ids; P.doc_chunk_off = a.doc_chunk_off; P.n_docs = a.n_docs; P.top_k = a.top_k;
+  P.max_sel = a.max_sel;
+  if (sh.list) {
+    P.sel_off = reinterpret_cast<const int64_t*>(w + L.list_off);
+    P.sel_chunk = reinterpret_cast<const int64_t*>(w + L.list_chunk);
+  }
+  P.rot_in_kernel = sh.rot ? 1 : 0;
+  P.rope_q = sh.dec ? 0 : 1;
   P.qrot = reinterpret_cast<float*>(w + L.qrot);
   P.krot = reinterpret_cast<float*>(w + L.krot);
   P.part_o = reinterpret_cast<float*>(w + L.part_o);
   P.part_ml = reinterpret_cast<float2*>(w + L.part_ml);
-  P.tickets = reinterpret_cast<unsigned*>(w + L.tickets);
+  P.tickets = sh.dec ? nullptr : reinterpret_cast<unsigned*>(w + L.tickets);  // the decoding kernel merges in a cluster
   P.out = a.out; P.out_f32 = a.out_f32; P.lse = a.lse;
   P.n_seq = a.n_seq; P.n_q = a.n_q; P.n_loc = sh.n_loc; P.hq = a.hq; P.hkv = a.hkv;
   P.group = a.hq / a.hkv; P.rt = sh.rt; P.n_splits = sh.n_splits; P.n_tiles = sh.n_tiles;
-  P.krot_split = (sh.dec || sh.tc) ? 1 : 0;
+  P.krot_split = (sh.tc || sh.dec) ? 1 : 0;
   P.scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)kHeadDim);
   P.pos_offset = (double)a.pos_offset;
   P.log2_theta = log2((double)a.rope_theta);
@@ -875,9 +904,10 @@ void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, cha
 
 msa_status launch_rope(const AttnParams& P, const msa_attend_args& a, const Shape& sh, cudaStream_t st) {
   const int gq = (a.hq + kRopeHeads - 1) / kRopeHeads, gk = (a.hkv + kRopeHeads - 1) / kRopeHeads;
-  int64_t n = (int64_t)a.n_q * gq * 64 + (int64_t)sh.n_loc * gk * 64;
-  const int64_t nt = (int64_t)sh.n_tiles * a.hkv;
+  int64_t n = (P.rope_q ? (int64_t)a.n_q * gq * 64 : 0) + (int64_t)sh.n_loc * gk * 64;
+  const int64_t nt = P.tickets ? (int64_t)sh.n_tiles * a.hkv : 0;
   if (n < nt) n = nt;
+  if (n < 1) n = 1;
   cudaError_t e = launch_pdl(rope_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: rotate queries and local keys");
   return launch_check("attend: rotate queries and local keys");
@@ -901,12 +931,24 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
   const Shape sh = plan(a, true);
   const Layout L = layout(a, sh);
   AttnParams P{};  // kernel parameter block (4.3 KB: large kernel parameters, CUDA >= 12.1)
-  fill_params(a, sh, L, reinterpret_cast<char*>(ws), P);
-  msa_status s = launch_rope(P, a, sh, st);
+  char* w = reinterpret_cast<char*>(ws);
+  fill_params(a, sh, L, w, P);
+  msa_status s = MSA_OK;
+  if (sh.list) {
+    s = launch_gather_index(a.doc_chunk_off, a.n_docs, a.top_ids, a.n_seq, a.top_k,
+                            reinterpret_cast<int64_t*>(w + L.list_off), reinterpret_cast<int64_t*>(w + L.list_chunk),
+                            (int64_t)a.n_seq * a.max_sel, st);
+    if (s != MSA_OK) return s;
+  }
+  if (sh.dec && sh.rot) return launch_attend_dec(P, st);  // rotates its own queries and local keys
+  if (sh.dec) {  // rope_rows rotates the local keys, the kernel its queries
+    s = launch_rope(P, a, sh, st);
+    return s != MSA_OK ? s : launch_attend_dec(P, st);
+  }
+  s = launch_rope(P, a, sh, st);
   if (s != MSA_OK) return s;
   if (sh.tc) return launch_attend_tc(P, st);
   if (g_attend_kernel == 3) return launch_attend_dec_tc(P, st);
-  if (sh.dec) return launch_attend_dec(P, sh.vec, st);
   dim3 grid((unsigned)sh.n_splits, (unsigned)a.hkv, (unsigned)sh.n_tiles);
   switch (sh.vec) {
     case 4: return launch_vec<4>(P, grid, st);
@@ -979,5 +1021,15 @@ extern "C" int msa_debug_set_attend_kernel(int which) {
 extern "C" int msa_debug_set_attend_splits(int n) {
   const int old = msa::g_attend_splits;
   if (n >= 0 && n <= 64) msa::g_attend_splits = n;
+  return old;
+}
+
+// Largest share of a sequence's local keys (per CTA) that the decoding kernel
+// rotates itself in later msa_attend calls (0..256; 0: rope_rows always does);
+// returns the previous setting. Workspace sizes follow the setting. A testing
+// and benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_dec_rot_keys(int n) {
+  const int old = msa::g_dec_rot_keys;
+  if (n >= 0 && n <= msa::kDecRotKeysMax) msa::g_dec_rot_keys = n;
   return old;
 }

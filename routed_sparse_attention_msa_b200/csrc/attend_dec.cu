@@ -10,25 +10,35 @@
 // few hundred keys per head (a few MB per layer at 4 flop per byte), so its
 // time is the chain of dependent memory round trips plus the latency of the
 // instructions each warp issues; neither bandwidth nor arithmetic throughput
-// bounds it. The kernel keeps that chain short:
+// bounds it. The kernel keeps that chain short, and is the call's only kernel:
 //  - A CTA (one per SM) owns one kv head, one tile of query vectors and one
 //    split of the key list: an even share of the sequence's memory keys (the
-//    selected pooled rows) and of its local keys (the recent context, rotated
-//    by rope_rows and stored there as bf16 high and low halves).
+//    selected pooled rows) and of its local keys (the recent context).
+//  - The CTA rotates its own query vectors (global positions offset by k),
+//    and, when its share of the local keys is small, those keys too, as bf16
+//    high and low halves (so the logits keep fp32 accuracy) while the first
+//    memory rows are already in flight. Local steps come first, so those keys
+//    go straight into the shared-memory stages that will compute them. A
+//    larger share is rotated before the kernel by rope_rows (a kernel of its
+//    own that spreads the work over the whole GPU) and copied like the rest.
+//    In the routed form the CTA lists the memory rows itself: the chunk
+//    ranges of the sequence's selected documents, scanned in shared memory.
 //  - Inside the CTA every warp is an independent flash-decoding worker: the
 //    share is cut into steps of 16 keys and warp w takes steps w, w + 8, ...
 //    Each warp copies its own steps' rows by cp.async into its own two
 //    shared-memory stages (the next step in flight while one is computed; a
-//    key's bank row is read from the selection list a step before its copy),
-//    keeps its own running max, sum and output, and synchronises with no
-//    other warp until the end.
+//    key's bank row is looked up a step before its copy), keeps its own
+//    running max, sum and output, and synchronises with no other warp until
+//    the end.
 //  - A step is two warp-level bf16 MMA chains (m16n8k16, fp32 accumulate), the
 //    16-vector tile as M: S = Q K^T (queries split into bf16 high + low parts,
-//    local keys too, so the logits keep fp32 accuracy), then O += P V with P
-//    taken straight from S's accumulators as the A operand (rounded to bf16).
-//  - At the end the 8 warps' (o, m, l) are merged through shared memory; with
-//    several splits per (tile, kv head) each CTA then writes an unnormalised
-//    partial and the last to finish (atomic ticket, no waiting) merges them.
+//    local keys too), then O += P V with P taken straight from S's
+//    accumulators as the A operand (rounded to bf16).
+//  - At the end the 8 warps' (o, m, l) are merged through shared memory; the
+//    splits of a (tile, kv head) are one thread-block cluster, whose CTAs then
+//    share out the outputs and merge the splits' partials by log-sum-exp
+//    straight from each other's shared memory (no partials in HBM, no
+//    counters to clear between calls).
 #include <math.h>
 
 #include "attend_params.cuh"
@@ -55,7 +65,13 @@ constexpr int kMRow = kHeadDim + 4;
 constexpr int offMO = 0;
 constexpr int offMM = offMO + kDWarps * kTileV * kMRow * 4;
 constexpr int offMLs = offMM + kDWarps * kTileV * 4;
-static_assert(offMLs + kDWarps * kTileV * 4 <= offQhi, "the merge fits the stages");
+// then this CTA's merged partial for the cluster merge: o [16][128] (unnormalised), m, l [16]
+constexpr int offPO = offMLs + kDWarps * kTileV * 4;
+constexpr int offPM = offPO + kTileV * kHeadDim * 4;
+constexpr int offPL = offPM + kTileV * 4;
+static_assert(offPL + kTileV * 4 <= offQhi, "the merge fits the stages");
+constexpr int kLocRowB = 2 * kHeadDim * 2;  // a local key rotated by rope_rows: high, then low halves
+constexpr int kRotBatch = 4;                // local-key rotations per thread whose loads go out first
 static_assert(kDecSmem <= 227 * 1024, "shared memory per CTA");
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -83,11 +99,54 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float bf_round_f(float x) { return __uint_as_float(f2bf_bits(x) << 16); }
+// Two floats to bf16 (round to nearest even) in one conversion: lo in bits 0-15, hi in 16-31.
+__device__ __forceinline__ uint32_t cvt_bf2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// x split into bf16 parts: x ~ h + l, h = bf16(x), l = bf16(x - h); a pair per call, packed.
+__device__ __forceinline__ void split_bf2(float x0, float x1, uint32_t& h, uint32_t& l) {
+  h = cvt_bf2(x0, x1);
+  l = cvt_bf2(x0 - bf_lo(h), x1 - bf_hi(h));
+}
+
+// ---- thread-block cluster: the splits of one (tile, kv head)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a float in the shared memory of cluster CTA `rank`, at this CTA's address `local` of the same variable
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local, uint32_t rank) {
+  uint32_t a;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+
+// RoPE of one pair (x0 = dim i, x1 = dim i + 64) at position pos (pair frequency f). The
+// angle is formed and reduced to [-pi, pi] in double; on that range the hardware sine and
+// cosine (__sincosf) are within 2^-21.4 absolute, well under the 2^-17 relative precision of
+// the bf16 high + low parts the results are stored in.
+__device__ __forceinline__ void rope_pair(float x0, float x1, double pos, double f, float& y0, float& y1) {
+  float sn, cs;
+  __sincosf(reduced_angle(pos * f), &sn, &cs);
+  y0 = x0 * cs - x1 * sn;
+  y1 = x0 * sn + x1 * cs;
+}
 
 __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ int s_last;
+  __shared__ int64_t s_pre[kDecRoutedMaxK + 1];  // routed form: first list position of each document
+  __shared__ int64_t s_c0[kDecRoutedMaxK];       // ... and its first chunk
+  __shared__ int64_t s_wsum[kDWarps];
+  __shared__ double s_invf[kHeadDim / 2];         // RoPE frequency of each pair
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, c = lane & 3;  // MMA fragment coordinates
@@ -105,50 +164,108 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   const int ga = g < nvec ? g0 + g / p.group : -1;
   const int gb = g + 8 < nvec ? g0 + (g + 8) / p.group : -1;
 
-  pdl_wait();  // the selection (gather) and the rotated rows (rope_rows) come from earlier kernels
+  pdl_wait();  // the selection comes from an earlier kernel
   pdl_trigger();
 
-  // ---- query tile (16 vectors v = rr * group + gg; past nvec zero): its loads go out
-  // together with those of the key ranges below
-  const int qv_v = tid >> 4, qv_d0 = 8 * (tid & 15);
-  float4 qa = make_float4(0.f, 0.f, 0.f, 0.f), qb = qa;
-  if (qv_v < nvec) {
-    const int rr = qv_v / p.group, gg = qv_v - rr * p.group;
-    const float4* qv = reinterpret_cast<const float4*>(
-        p.qrot + ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim + qv_d0);
-    qa = __ldcg(qv);
-    qb = __ldcg(qv + 1);
-  }
-
-  // ---- this split's share of the memory keys [m0, m1) and of the local keys [l0, l1)
-  const int64_t mem_base = __ldcg(p.sel_off + s);
-  const int64_t n_mem = __ldcg(p.sel_off + s + 1) - mem_base;
-  const int64_t pm = (n_mem + p.n_splits - 1) / p.n_splits;
-  const int64_t m0 = min(n_mem, (int64_t)sp * pm), m1 = min(n_mem, m0 + pm);
+  // ---- this split's share of the local keys [l0, l1) (known from the host's offsets): local
+  // steps come first, so that a CTA's first 16 local steps are its warps' first two steps and
+  // their rotated keys go straight into those stages
   const int pl = (lvis + p.n_splits - 1) / p.n_splits;
   const int l0 = min(lvis, sp * pl), l1 = min(lvis, l0 + pl);
-  const int nsm = (int)((m1 - m0 + kStepKeys - 1) / kStepKeys);  // memory steps, then local steps
-  const int nsteps = nsm + (l1 - l0 + kStepKeys - 1) / kStepKeys;
+  const int nsl = (l1 - l0 + kStepKeys - 1) / kStepKeys;  // local steps
 
-  // ---- this warp's steps w, w + 8, ...: lane kl < 16 looks up the bank row of key kl of a
-  // step; copy instruction u then moves rows 2u and 2u + 1 whole (lanes 0-15 and 16-31, 16 B
-  // each), so every instruction reads two contiguous 256-byte rows
+  // loads that depend on nothing in flight go out first: the query tile (16 vectors
+  // v = rr * group + gg, past nvec zero; thread -> vector qv_v, dims qv_d0 .. qv_d0 + 7, its
+  // rotation partners, dims +- 64, held by lane ^ 8), the first batch of the local keys to
+  // rotate (thread -> key, dims 2j, 2j + 1 and their partners + 64), and the frequencies
+  if (tid < kHeadDim / 2) s_invf[tid] = p.inv_freq[tid];
+  const int qv_v = tid >> 4, qv_d0 = 8 * (tid & 15);
+  uint4 qraw = make_uint4(0, 0, 0, 0);
+  if (qv_v < nvec) {
+    const int rr = qv_v / p.group, gg = qv_v - rr * p.group;
+    qraw = __ldcg(reinterpret_cast<const uint4*>(p.q + ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim +
+                                                 qv_d0));
+  }
+  const int nrot = p.rot_in_kernel ? (l1 - l0) * 32 : 0;  // at most 16 steps' keys (the host sees to it)
+  auto kloc_ptr = [&](int it) {
+    return p.k_loc + ((size_t)(p.loc_off[s] + l0 + (it >> 5)) * p.hkv + kvh) * kHeadDim + 2 * (it & 31);
+  };
+  uint32_t ka[kRotBatch], kb2[kRotBatch];
+#pragma unroll
+  for (int u = 0; u < kRotBatch; ++u) {
+    const int it = tid + u * kDThreads;
+    if (it < nrot) {
+      ka[u] = __ldcg(reinterpret_cast<const unsigned int*>(kloc_ptr(it)));
+      kb2[u] = __ldcg(reinterpret_cast<const unsigned int*>(kloc_ptr(it) + 64));
+    }
+  }
+
+  // ---- the sequence's memory rows: the gather listing (sel_off, sel_chunk), or in the
+  // routed form the chunks of its selected documents in rank order
+  const bool routed = p.sel_off == nullptr;
+  int64_t mem_base = 0, n_mem;
+  if (routed) {
+    int64_t c0 = 0, cnt = 0;
+    if (tid < p.top_k) {
+      const int32_t doc = __ldcg(p.top_ids + (size_t)s * p.top_k + tid);
+      if (doc >= 0 && doc < p.n_docs) {
+        c0 = __ldcg(p.doc_chunk_off + doc);
+        cnt = __ldcg(p.doc_chunk_off + doc + 1) - c0;
+      }
+    }
+    int64_t x = cnt;  // inclusive scan over the block (top_k <= 256 = its threads)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wsum[w] = x;
+    __syncthreads();
+    for (int j = 0; j < w; ++j) x += s_wsum[j];
+    if (tid < p.top_k) {
+      s_pre[tid] = x - cnt;
+      s_c0[tid] = c0;
+    }
+    if (tid == p.top_k - 1) s_pre[p.top_k] = x;
+    __syncthreads();
+    n_mem = min(s_pre[p.top_k], p.max_sel);
+  } else {
+    mem_base = __ldcg(p.sel_off + s);
+    n_mem = __ldcg(p.sel_off + s + 1) - mem_base;
+  }
+
+  // ---- this split's share of the memory keys [m0, m1): the steps after the local ones
+  const int64_t pm = (n_mem + p.n_splits - 1) / p.n_splits;
+  const int64_t m0 = min(n_mem, (int64_t)sp * pm), m1 = min(n_mem, m0 + pm);
+  const int nsteps = nsl + (int)((m1 - m0 + kStepKeys - 1) / kStepKeys);
+
+  // ---- this warp's steps w, w + 8, ...: lane kl < 16 looks up the row of key kl of a step;
+  // copy instruction u then moves rows 2u and 2u + 1 whole (lanes 0-15 and 16-31, 16 B each),
+  // so every instruction reads two contiguous 256-byte rows
   const int kl = lane & 15;
   uint8_t* wst = sm + w * kWarpB;
-  auto row_of = [&](int i) -> int64_t {  // bank row (memory) or local row of key kl in step i; -1: none
+  auto row_of = [&](int i) -> int64_t {  // local key or bank row (memory) of key kl in step i; -1: none
     if (i >= nsteps) return -1;
-    if (i < nsm) {
-      const int64_t key = m0 + (int64_t)i * kStepKeys + kl;
-      if (key >= m1) return -1;
-      return p.sel_chunk ? __ldcg(p.sel_chunk + mem_base + key) : mem_base + key;
+    if (i < nsl) {
+      const int key = l0 + i * kStepKeys + kl;
+      return key < l1 ? (int64_t)key : -1;
     }
-    const int key = l0 + (i - nsm) * kStepKeys + kl;
-    return key < l1 ? (int64_t)(p.loc_off[s] + key) : -1;
+    const int64_t key = m0 + (int64_t)(i - nsl) * kStepKeys + kl;
+    if (key >= m1) return -1;
+    if (!routed) return p.sel_chunk ? __ldcg(p.sel_chunk + mem_base + key) : mem_base + key;
+    int lo = 0, hi = p.top_k - 1;  // the last document whose first list position is <= key
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= key) lo = mid; else hi = mid - 1;
+    }
+    return s_c0[lo] + (key - s_pre[lo]);
   };
-  auto issue = [&](int i, int64_t r_mine, int stage) {
+  // k_in_place: the step's local keys are rotated straight into the stage (the warp's first two
+  // steps in the in-kernel rotation mode, which has at most 16 local steps), so only V is copied
+  auto issue = [&](int i, int64_t r_mine, int stage, bool k_in_place) {
     if (i < nsteps) {
       uint8_t* stg = wst + stage * kStageB;
-      const bool loc = i >= nsm;
+      const bool loc = i < nsl;
       const int piece = 16 * (lane & 15);
 #pragma unroll
       for (int u = 0; u < kStepKeys / 2; ++u) {
@@ -161,10 +278,12 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
             cp16(saddr(stg + offSK + so), reinterpret_cast<const uint8_t*>(p.mem_k) + off);
             cp16(saddr(stg + offSV + so), reinterpret_cast<const uint8_t*>(p.mem_v) + off);
           } else {
-            const size_t lrow = (size_t)r * p.hkv + kvh;
-            const uint8_t* kr = reinterpret_cast<const uint8_t*>(p.krot) + lrow * 512;  // high, then low halves
-            cp16(saddr(stg + offSK + so), kr + piece);
-            cp16(saddr(stg + offSL + so), kr + 256 + piece);
+            const size_t lrow = (size_t)(p.loc_off[s] + r) * p.hkv + kvh;
+            if (!k_in_place) {  // rotated by rope_rows
+              const uint8_t* kr = reinterpret_cast<const uint8_t*>(p.krot) + lrow * kLocRowB;  // high, then low
+              cp16(saddr(stg + offSK + so), kr + piece);
+              cp16(saddr(stg + offSL + so), kr + 256 + piece);
+            }
             cp16(saddr(stg + offSV + so), reinterpret_cast<const uint8_t*>(p.v_loc + lrow * kHeadDim) + piece);
           }
         } else {
@@ -175,29 +294,67 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     }
     cp_commit();
   };
-  int64_t r_next;  // bank row of key kl in the warp's third step
   {
-    const int64_t r0 = row_of(w), r1 = row_of(w + kDWarps), r2 = row_of(w + 2 * kDWarps);
-    issue(w, r0, 0);
-    issue(w + kDWarps, r1, 1);
-    r_next = r2;
+    const int64_t r0 = row_of(w), r1 = row_of(w + kDWarps);
+    issue(w, r0, 0, p.rot_in_kernel);
+    issue(w + kDWarps, r1, 1, p.rot_in_kernel);
   }
+  int64_t r_next = row_of(w + 2 * kDWarps);  // row of key kl in the warp's third step
+  __syncthreads();  // the frequencies
 
-  // ---- queries as bf16 high and low parts (shared by the warps)
-  {
-    const float f[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-    float h[8], l[8];
+  // ---- rotate this CTA's local keys (global positions pos_offset + j) into bf16 high and low
+  // halves, local step j straight into stage j / 8 of warp j % 8 (j < 16)
+  auto rotate_store = [&](int it, uint32_t a, uint32_t b) {
+    const int jl = it >> 5, i = 2 * (it & 31);
+    const double pos = p.pos_offset + (double)(l0 + jl);
+    float y0a, y1a, y0b, y1b;
+    rope_pair(bf_lo(a), bf_lo(b), pos, s_invf[i], y0a, y1a);
+    rope_pair(bf_hi(a), bf_hi(b), pos, s_invf[i + 1], y0b, y1b);
+    uint32_t hi0, lo0, hi1, lo1;
+    split_bf2(y0a, y0b, hi0, lo0);
+    split_bf2(y1a, y1b, hi1, lo1);
+    const int step = jl / kStepKeys;
+    uint8_t* row = sm + (step % kDWarps) * kWarpB + (step / kDWarps) * kStageB + (jl % kStepKeys) * kRowB;
+    *reinterpret_cast<uint32_t*>(row + offSK + 2 * i) = hi0;
+    *reinterpret_cast<uint32_t*>(row + offSK + 2 * (64 + i)) = hi1;
+    *reinterpret_cast<uint32_t*>(row + offSL + 2 * i) = lo0;
+    *reinterpret_cast<uint32_t*>(row + offSL + 2 * (64 + i)) = lo1;
+  };
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[i] = bf_round_f(f[i]);
-      l[i] = f[i] - h[i];
-    }
-    *reinterpret_cast<uint4*>(sm + offQhi + qv_v * kRowB + 2 * qv_d0) =
-        make_uint4(pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]), pack_bf2(h[6], h[7]));
-    *reinterpret_cast<uint4*>(sm + offQlo + qv_v * kRowB + 2 * qv_d0) =
-        make_uint4(pack_bf2(l[0], l[1]), pack_bf2(l[2], l[3]), pack_bf2(l[4], l[5]), pack_bf2(l[6], l[7]));
+  for (int u = 0; u < kRotBatch; ++u) {
+    const int it = tid + u * kDThreads;
+    if (it < nrot) rotate_store(it, ka[u], kb2[u]);
   }
-  __syncthreads();
+  for (int it = tid + kRotBatch * kDThreads; it < nrot; it += kDThreads) {
+    const uint32_t a = __ldcg(reinterpret_cast<const unsigned int*>(kloc_ptr(it)));
+    const uint32_t b = __ldcg(reinterpret_cast<const unsigned int*>(kloc_ptr(it) + 64));
+    rotate_store(it, a, b);
+  }
+  // ---- queries, rotated, as bf16 high and low parts (shared by the warps)
+  {
+    uint32_t mine[4] = {qraw.x, qraw.y, qraw.z, qraw.w}, other[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) other[e] = __shfl_xor_sync(0xffffffffu, mine[e], 8);
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (qv_v < nvec) {
+      const double pos = p.pos_offset + (double)(g0 + qv_v / p.group);
+      const bool first = qv_d0 < 64;  // this thread holds x0 (dims < 64) or x1 (dims >= 64) of its pairs
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float xm = (e & 1) ? bf_hi(mine[e >> 1]) : bf_lo(mine[e >> 1]);
+        const float xo = (e & 1) ? bf_hi(other[e >> 1]) : bf_lo(other[e >> 1]);
+        float y0, y1;
+        rope_pair(first ? xm : xo, first ? xo : xm, pos, s_invf[(qv_d0 & 63) + e], y0, y1);
+        y[e] = first ? y0 : y1;
+      }
+    }
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_bf2(y[2 * i], y[2 * i + 1], h[i], l[i]);
+    *reinterpret_cast<uint4*>(sm + offQhi + qv_v * kRowB + 2 * qv_d0) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(sm + offQlo + qv_v * kRowB + 2 * qv_d0) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+  __syncthreads();  // the query parts and the local keys written in place
 
   // Q as the A operand of S, all 8 k-steps (16 dims each), high and low parts: held in
   // registers for every step of the warp
@@ -230,8 +387,8 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     cp_wait<1>();  // this step's copies (this lane's); the next step's may still be in flight
     __syncwarp();  // ... and every lane's
     const uint8_t* stg = wst + stage * kStageB;
-    const bool loc = i >= nsm;
-    const int64_t kb = loc ? l0 + (int64_t)(i - nsm) * kStepKeys : m0 + (int64_t)i * kStepKeys;
+    const bool loc = i < nsl;
+    const int64_t kb = loc ? l0 + (int64_t)i * kStepKeys : m0 + (int64_t)(i - nsl) * kStepKeys;
     const int nk = (int)min((int64_t)kStepKeys, (loc ? l1 : m1) - kb);
 
     // ---- S (16 vectors x 16 keys) = Q K^T: n-tiles 0 (keys 0-7) and 1 (keys 8-15), each
@@ -302,8 +459,8 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     mA = nA;
     mB = nB;
     // P as the A operand of P.V (16 vectors x 16 keys): the accumulator layout of S's two n-tiles
-    const uint32_t pa[4] = {pack_bf2(pr[0][0], pr[0][1]), pack_bf2(pr[0][2], pr[0][3]), pack_bf2(pr[1][0], pr[1][1]),
-                            pack_bf2(pr[1][2], pr[1][3])};
+    const uint32_t pa[4] = {cvt_bf2(pr[0][0], pr[0][1]), cvt_bf2(pr[0][2], pr[0][3]), cvt_bf2(pr[1][0], pr[1][1]),
+                            cvt_bf2(pr[1][2], pr[1][3])};
 
     // ---- O = O * corr + P V over the 128 dims (16 n-tiles of 8); most steps leave the max in place
     if (__any_sync(0xffffffffu, cA != 1.f || cB != 1.f)) {
@@ -322,7 +479,7 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     }
     __syncwarp();  // every lane is done with this stage
     // the warp's step after next goes into this stage
-    issue(i + 2 * kDWarps, r_next, stage);
+    issue(i + 2 * kDWarps, r_next, stage, false);
     r_next = row_of(i + 3 * kDWarps);
   }
   cp_wait<0>();
@@ -347,6 +504,9 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   __syncthreads();
   const int d = tid & (kHeadDim - 1);
   const bool split = p.n_splits > 1;
+  float* po = reinterpret_cast<float*>(sm + offPO);
+  float* pm_ = reinterpret_cast<float*>(sm + offPM);
+  float* pl_ = reinterpret_cast<float*>(sm + offPL);
   for (int v = tid >> 7; v < nvec; v += 2) {
     float m = -INFINITY;
 #pragma unroll
@@ -360,59 +520,88 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
         r += mo[(x * kTileV + v) * kMRow + d] * wt;
       }
     }
-    const int rr = v / p.group, gg = v - rr * p.group;
-    const size_t rh = (size_t)(row0 + rr) * p.hq + kvh * p.group + gg;
     if (!split) {
+      const int rr = v / p.group, gg = v - rr * p.group;
+      const size_t rh = (size_t)(row0 + rr) * p.hq + kvh * p.group + gg;
       const float res = l > 0.f ? r / l : 0.f;
       p.out[rh * kHeadDim + d] = (uint16_t)f2bf_bits(res);
       if (p.out_f32) p.out_f32[rh * kHeadDim + d] = res;
       if (p.lse && d == 0) p.lse[rh] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
-      const size_t pi = rh * p.n_splits + sp;
-      p.part_o[pi * kHeadDim + d] = r;
-      if (d == 0) p.part_ml[pi] = make_float2(m, l);
+      po[v * kHeadDim + d] = r;
+      if (d == 0) {
+        pm_[v] = m;
+        pl_[v] = l;
+      }
     }
   }
   if (!split) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(p.tickets + (size_t)tile * p.hkv + kvh, 1u) == (unsigned)(p.n_splits - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // ---- the last CTA of this (tile, kv head) merges every split (log2 units)
-  for (int v = tid >> 7; v < nvec; v += 2) {
-    const int rr = v / p.group, gg = v - rr * p.group;
-    const size_t rh = (size_t)(row0 + rr) * p.hq + kvh * p.group + gg;
-    float mx = -INFINITY;
-    for (int j = 0; j < p.n_splits; ++j) {
-      const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
-      if (x.y > 0.f) mx = fmaxf(mx, x.x);
+  // ---- the cluster merges its splits' partials (log2 units) straight from their shared
+  // memory: output (v, d) number o goes to CTA o / 256 mod splits, each thread loading all
+  // splits' values at once; the second barrier keeps every CTA's memory alive until then
+  cluster_sync();
+  {
+    const int ns = p.n_splits;
+    const int rank = (int)cluster_rank();
+    for (int o = rank * kDThreads + tid; o < nvec * kHeadDim; o += ns * kDThreads) {
+      const int v = o / kHeadDim, dd = o % kHeadDim;
+      float lj[kDecMaxSplits], mj[kDecMaxSplits], oj[kDecMaxSplits];
+#pragma unroll
+      for (int j = 0; j < kDecMaxSplits; ++j) {
+        lj[j] = 0.f;
+        mj[j] = -INFINITY;
+        oj[j] = 0.f;
+        if (j < ns) {
+          lj[j] = ld_cluster_f32(saddr(pl_ + v), j);
+          mj[j] = ld_cluster_f32(saddr(pm_ + v), j);
+          oj[j] = ld_cluster_f32(saddr(po + v * kHeadDim + dd), j);
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kDecMaxSplits; ++j)
+        if (lj[j] > 0.f) mx = fmaxf(mx, mj[j]);
+      float wsum = 0.f, r = 0.f;
+#pragma unroll
+      for (int j = 0; j < kDecMaxSplits; ++j) {
+        if (lj[j] > 0.f) {
+          const float wt = exp2f(mj[j] - mx);
+          wsum += lj[j] * wt;
+          r += wt * oj[j];
+        }
+      }
+      r = wsum > 0.f ? r / wsum : 0.f;
+      const int rr = v / p.group, gg = v - rr * p.group;
+      const size_t rh = (size_t)(row0 + rr) * p.hq + kvh * p.group + gg;
+      p.out[rh * kHeadDim + dd] = (uint16_t)f2bf_bits(r);
+      if (p.out_f32) p.out_f32[rh * kHeadDim + dd] = r;
+      if (p.lse && dd == 0) p.lse[rh] = wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
     }
-    float wsum = 0.f, r = 0.f;
-    for (int j = 0; j < p.n_splits; ++j) {
-      const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
-      if (!(x.y > 0.f)) continue;
-      const float wt = exp2f(x.x - mx);
-      wsum += x.y * wt;
-      r += wt * __ldcg(p.part_o + (rh * p.n_splits + j) * kHeadDim + d);
-    }
-    r = wsum > 0.f ? r / wsum : 0.f;
-    p.out[rh * kHeadDim + d] = (uint16_t)f2bf_bits(r);
-    if (p.out_f32) p.out_f32[rh * kHeadDim + d] = r;
-    if (p.lse && d == 0) p.lse[rh] = wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
   }
+  cluster_sync();
 }
 
 }  // namespace
 
-msa_status launch_attend_dec(const AttnParams& P, int vec, cudaStream_t st) {
-  (void)vec;  // the tile is always 16 MMA rows; P.rt rows x P.group heads of them are used
+msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st) {
   static std::atomic<uint64_t> attr{0};
   cudaError_t e = smem_limit_once(attend_dec_kernel, kDecSmem, attr);
   if (e != cudaSuccess) return cuda_fail(e, "attend: decoding kernel shared memory");
-  e = launch_pdl(attend_dec_kernel, dim3((unsigned)P.n_splits, (unsigned)P.hkv, (unsigned)P.n_tiles),
-                 dim3(kDThreads), (size_t)kDecSmem, st, P);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P.n_splits, (unsigned)P.hkv, (unsigned)P.n_tiles);
+  cfg.blockDim = dim3(kDThreads);
+  cfg.dynamicSmemBytes = (size_t)kDecSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;  // the splits of a (tile, kv head): one cluster
+  at[1].val.clusterDim.x = (unsigned)P.n_splits;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = P.n_splits > 1 ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, attend_dec_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: decoding kernel");
   return launch_check("attend: decoding kernel");
 }

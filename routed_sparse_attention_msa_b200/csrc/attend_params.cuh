@@ -13,10 +13,16 @@ struct AttnParams {
   const uint16_t* v_loc;
   const uint16_t* mem_k;
   const uint16_t* mem_v;
-  const int64_t* sel_off;
+  const int64_t* sel_off;        // nullptr: the routed form below
   const int64_t* sel_chunk;
+  const int32_t* top_ids;        // routed form: [n_seq, top_k] selected documents
+  const int64_t* doc_chunk_off;  // routed form: [n_docs + 1] each document's chunk range
+  int64_t n_docs, max_sel;
+  int top_k;
+  int rot_in_kernel;  // decoding kernel: 1 = it rotates its local keys itself, 0 = rope_rows did
+  int rope_q;         // rope_rows: 1 = rotate the query rows too (0: the decoding kernel does)
   float* qrot;      // [n_q, hq, d]
-  float* krot;      // [n_loc, hkv, d]
+  float* krot;      // [n_loc, hkv, d], or [n_loc, hkv] rows of 512 B with krot_split
   float* part_o;    // [n_q, hq, splits, d]
   float2* part_ml;  // [n_q, hq, splits]
   unsigned* tickets;  // [n_tiles * hkv]
@@ -33,6 +39,14 @@ struct AttnParams {
   int32_t loc_off[kMaxSeq + 1];
   int32_t tile_off[kMaxSeq + 1];
 };
+
+// An angle (radians, double) reduced to [-pi, pi] in double, as a float: sincosf
+// then evaluates it on its short, accurate range for positions of any size.
+__device__ __forceinline__ float reduced_angle(double ang) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  return (float)(ang - two_pi * rint(ang * inv_two_pi));
+}
 
 // Index of the segment of `off` (n_seq + 1 ascending offsets) holding x.
 __device__ __forceinline__ int seq_of(const int32_t* off, int n_seq, int x) {
@@ -58,9 +72,15 @@ msa_status launch_attend_dec_tc(const AttnParams& P, cudaStream_t st);
 
 // attend_dec.cu: the decoding shapes (at most 16 query vectors per tile),
 // grid (n_splits, hkv, n_tiles), each split an even share of every
-// sequence's memory and local keys. Needs rope_rows to have run with
-// krot_split = 1.
-msa_status launch_attend_dec(const AttnParams& P, int vec, cudaStream_t st);
+// sequence's memory and local keys; the splits of a (tile, kv head) form one
+// cluster. It rotates its own queries, and its local keys too when each
+// CTA's share is at most kDecRotKeys (otherwise rope_rows rotates them first,
+// krot_split = 1, rope_q = 0); it lists the routed form's memory rows itself
+// when top_k <= kDecRoutedMaxK.
+constexpr int kDecMaxSplits = 8;
+constexpr int kDecRoutedMaxK = 256;
+constexpr int kDecRotKeysMax = 256;  // in-kernel rotation: the local keys of a CTA's first 16 steps at most
+msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st);
 int attend_dec_tc_error_take();
 
 }  // namespace msa

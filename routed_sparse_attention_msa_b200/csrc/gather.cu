@@ -18,9 +18,11 @@ namespace {
 // loop).
 constexpr int kIndexThreads = 1024;
 
+// An id outside [0, n_docs) lists no chunks; list positions from `cap` on are
+// not written (offsets are clamped to cap), so the list never leaves its buffer.
 __global__ void __launch_bounds__(kIndexThreads) gather_index_kernel(
-    const int64_t* __restrict__ doc_chunk_off, const int32_t* __restrict__ top_ids, int n_seq,
-    int k, int64_t* __restrict__ sel_off, int64_t* __restrict__ sel_chunk) {
+    const int64_t* __restrict__ doc_chunk_off, int64_t n_docs, const int32_t* __restrict__ top_ids, int n_seq,
+    int k, int64_t* __restrict__ sel_off, int64_t* __restrict__ sel_chunk, int64_t cap) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t s_start[kIndexThreads], s_c0[kIndexThreads];
   __shared__ int64_t carry;
@@ -35,8 +37,10 @@ __global__ void __launch_bounds__(kIndexThreads) gather_index_kernel(
     int64_t c0 = 0, n = 0;
     if (p < n_pairs) {
       const int32_t doc = __ldcg(top_ids + p);
-      c0 = doc_chunk_off[doc];
-      n = doc_chunk_off[doc + 1] - c0;
+      if (doc >= 0 && doc < n_docs) {
+        c0 = doc_chunk_off[doc];
+        n = doc_chunk_off[doc + 1] - c0;
+      }
     }
     int64_t x = n;
 #pragma unroll
@@ -61,12 +65,12 @@ __global__ void __launch_bounds__(kIndexThreads) gather_index_kernel(
     s_start[tid] = p < n_pairs ? start : INT64_MAX;
     s_c0[tid] = c0;
     if (p < n_pairs) {
-      if (p % k == 0) sel_off[p / k] = start;
-      if (p == n_pairs - 1) sel_off[n_seq] = start + n;
+      if (p % k == 0) sel_off[p / k] = min(start, cap);
+      if (p == n_pairs - 1) sel_off[n_seq] = min(start + n, cap);
     }
     const int64_t c_new = c_old + warp_sums[31];
     __syncthreads();
-    for (int64_t j = c_old + tid; j < c_new; j += kIndexThreads) {
+    for (int64_t j = c_old + tid; j < min(c_new, cap); j += kIndexThreads) {
       int lo = 0, hi = kIndexThreads - 1;  // the last pair whose start is <= j
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -126,10 +130,10 @@ __global__ void gather_pull_kernel(const uint16_t* __restrict__ kbar, const uint
 
 }  // namespace
 
-msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
-                               int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st) {
-  cudaError_t e = launch_pdl(gather_index_kernel, dim3(1), dim3(1024), 0, st, b.doc_chunk_off, top_ids, n_seq, k,
-                             sel_off, sel_chunk);
+msa_status launch_gather_index(const int64_t* doc_chunk_off, int64_t n_docs, const int32_t* top_ids, int n_seq,
+                               int k, int64_t* sel_off, int64_t* sel_chunk, int64_t cap, cudaStream_t st) {
+  cudaError_t e = launch_pdl(gather_index_kernel, dim3(1), dim3(1024), 0, st, doc_chunk_off, n_docs, top_ids, n_seq,
+                             k, sel_off, sel_chunk, cap);
   if (e != cudaSuccess) return cuda_fail(e, "gather: chunk list");
   return launch_check("gather: chunk list");
 }

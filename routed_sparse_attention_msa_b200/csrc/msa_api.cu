@@ -296,7 +296,7 @@ msa_status msa_gather(const msa_gather_args* a, void* stream) {
       return fail(MSA_ERR_INVALID_ARG, "gather: copy-engine mode needs doc_chunk_off_host, top_ids_host, copy_stream, done_event");
   }
   cudaStream_t st = (cudaStream_t)stream;
-  s = launch_gather_index(b, a->top_ids, a->n_seq, k, a->sel_off, a->sel_chunk, st);
+  s = launch_gather_index(b.doc_chunk_off, b.n_docs, a->top_ids, a->n_seq, k, a->sel_off, a->sel_chunk, a->cap, st);
   if (s != MSA_OK || !b.content_on_host) return s;
   if (a->mode == MSA_GATHER_DEVICE_PULL) {
     // The kernel reads the pinned host rows through their device-side mapping.
@@ -361,8 +361,16 @@ static msa_status check_attend(const msa_attend_args* a) {
   const int g = a->hq / a->hkv;
   if (g > 16 || (g & (g - 1))) return fail(MSA_ERR_UNSUPPORTED, "attend: hq / hkv = %d (1, 2, 4, 8 or 16)", g);
   if (a->n_seq <= 0 || a->n_seq > kMaxSeq) return fail(MSA_ERR_UNSUPPORTED, "attend: n_seq = %d (1..%d)", a->n_seq, kMaxSeq);
-  if (!a->q || !a->q_seq_off || !a->q_start || !a->loc_off || !a->sel_off || !a->out)
+  if (!a->q || !a->q_seq_off || !a->q_start || !a->loc_off || !a->out)
     return fail(MSA_ERR_INVALID_ARG, "attend: NULL pointer");
+  if (!a->sel_off == !a->top_ids)
+    return fail(MSA_ERR_INVALID_ARG, "attend: give exactly one of sel_off (a gather listing) and top_ids (routed)");
+  if (a->top_ids) {
+    if (a->sel_chunk) return fail(MSA_ERR_INVALID_ARG, "attend: routed form takes no sel_chunk");
+    if (!a->doc_chunk_off) return fail(MSA_ERR_INVALID_ARG, "attend: routed form needs doc_chunk_off");
+    if (a->top_k <= 0 || a->top_k > 4096) return fail(MSA_ERR_INVALID_ARG, "attend: top_k = %d (1..4096)", a->top_k);
+    if (a->n_docs < 0) return fail(MSA_ERR_INVALID_ARG, "attend: n_docs < 0");
+  }
   if (a->q_seq_off[0] != 0 || a->q_seq_off[a->n_seq] != a->n_q)
     return fail(MSA_ERR_INVALID_ARG, "attend: q_seq_off must start at 0 and end at n_q");
   if (a->loc_off[0] != 0) return fail(MSA_ERR_INVALID_ARG, "attend: loc_off[0] must be 0");
@@ -423,6 +431,7 @@ msa_status msa_route_backward(const msa_bank_layer* b, const uint16_t* qr, const
 msa_status msa_attend_backward_workspace(const msa_attend_args* a, size_t* bytes) {
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
+  if (a->top_ids) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: needs a gather listing (sel_off), not the routed form");
   if (!bytes) return fail(MSA_ERR_INVALID_ARG, "attend_backward_workspace: bytes is NULL");
   *bytes = attend_backward_workspace(*a);
   return MSA_OK;
@@ -432,6 +441,7 @@ msa_status msa_attend_backward(const msa_attend_args* a, const float* dout, floa
                                float* dmem_k, float* dmem_v, void* ws, size_t ws_bytes, void* stream) {
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
+  if (a->top_ids) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: needs a gather listing (sel_off), not the routed form");
   if (!a->out_f32 || !a->lse) return fail(MSA_ERR_INVALID_ARG, "attend_backward: the forward's out_f32 and lse are required");
   if (!dout || !dq) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dout or dq");
   if (a->loc_off[a->n_seq] > 0 && (!dk_loc || !dv_loc)) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dk_loc/dv_loc");

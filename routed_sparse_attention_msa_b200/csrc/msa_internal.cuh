@@ -157,8 +157,8 @@ msa_status launch_topk_merge(const int32_t* ids, const float* scores, const int6
                              int n_seq, int k, int k_out, int32_t* top_ids, float* top_scores, cudaStream_t st);
 
 // gather.cu
-msa_status launch_gather_index(const msa_bank_layer& b, const int32_t* top_ids, int n_seq, int k,
-                               int64_t* sel_off, int64_t* sel_chunk, cudaStream_t st);
+msa_status launch_gather_index(const int64_t* doc_chunk_off, int64_t n_docs, const int32_t* top_ids, int n_seq,
+                               int k, int64_t* sel_off, int64_t* sel_chunk, int64_t cap, cudaStream_t st);
 msa_status launch_gather_pull(const msa_bank_layer& b, const int64_t* sel_off,
                               const int64_t* sel_chunk, int64_t cap, uint16_t* stage_k,
                               uint16_t* stage_v, cudaStream_t st);

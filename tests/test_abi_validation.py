@@ -206,6 +206,15 @@ ATTEND_CASES = [
     (dict(max_sel=-1), INVALID, "max_sel"),
     (dict(mem_v=None), INVALID, "memory K/V"),
     (dict(rope_theta=1.0), INVALID, "rope_theta"),
+    # the routed form (top_ids instead of a gather listing)
+    (dict(top_ids=FAKE), INVALID, "exactly one"),
+    (dict(sel_off=None), INVALID, "exactly one"),
+    (dict(sel_off=None, top_ids=FAKE, doc_chunk_off=FAKE, n_docs=5, top_k=4), INVALID, "no sel_chunk"),
+    (dict(sel_off=None, sel_chunk=None, top_ids=FAKE, n_docs=5, top_k=4), INVALID, "doc_chunk_off"),
+    (dict(sel_off=None, sel_chunk=None, top_ids=FAKE, doc_chunk_off=FAKE, n_docs=5, top_k=0), INVALID, "top_k = 0"),
+    (dict(sel_off=None, sel_chunk=None, top_ids=FAKE, doc_chunk_off=FAKE, n_docs=5, top_k=5000), INVALID,
+     "top_k = 5000"),
+    (dict(sel_off=None, sel_chunk=None, top_ids=FAKE, doc_chunk_off=FAKE, n_docs=-1, top_k=4), INVALID, "n_docs"),
 ]
 
 
@@ -234,6 +243,17 @@ def test_attend_valid_arguments_need_a_workspace(msa):
     # no query rows: nothing to do, nothing enqueued
     z, keep2 = _attend(msa, q_seq_off=[0, 0], n_q=0)
     assert msa._lib.msa_attend(ctypes.byref(z), FAKE, 1 << 30, None) == 0
+
+
+@host_only
+def test_attend_routed_form_is_forward_only(msa):
+    a, keep = _attend(msa, sel_off=None, sel_chunk=None, top_ids=FAKE, doc_chunk_off=FAKE, n_docs=5, top_k=4)
+    n = ctypes.c_size_t()
+    assert msa._lib.msa_attend_workspace(ctypes.byref(a), ctypes.byref(n)) == 0 and n.value > 0
+    assert msa._lib.msa_attend_backward_workspace(ctypes.byref(a), ctypes.byref(n)) == UNSUPPORTED
+    assert msa._lib.msa_attend_backward(ctypes.byref(a), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                        None) == UNSUPPORTED
+    assert "routed form" in _last(msa)
 
 
 @host_only

@@ -367,10 +367,14 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc", "tc_dec", "dec"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope"])
 def attend_kernel(request, msa):
-    old = msa.set_attend_kernel(request.param)
+    """dec: the decoding kernel rotating its local keys itself; dec_rope: the
+    same kernel after the separate rotation kernel."""
+    old = msa.set_attend_kernel(request.param.replace("_rope", ""))
+    old_r = msa.set_dec_rot_keys(0 if request.param == "dec_rope" else 256)
     yield request.param
+    msa.set_dec_rot_keys(old_r)
     msa.set_attend_kernel(old)
 
 
@@ -453,18 +457,21 @@ def test_attend_staged_memory_equals_indexed(msa, attend_kernel):
     np.testing.assert_array_equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("kernel", ["split", "dec"])
+@pytest.mark.parametrize("kernel", ["split", "dec", "dec_rope"])
 @pytest.mark.parametrize("splits", [1, 2, 5, 64])
 def test_attend_forced_splits(msa, kernel, splits):
     """Key splits forced (split-K: 64 is clamped to one split per 32 keys;
-    decoding kernel: the memory-key CTAs, at least 64 keys each, so one or two
-    splits walk several pipelined blocks): splits that get no keys, one split,
-    uneven splits."""
-    old_k, old_s = msa.set_attend_kernel(kernel), msa.set_attend_splits(splits)
+    decoding kernel: 64 is clamped to its 8-CTA cluster, with one split a CTA
+    walks every key of its sequence): splits that get no keys, one split,
+    uneven splits; the decoding kernel rotating its local keys itself or after
+    the separate rotation kernel."""
+    old_k, old_s = msa.set_attend_kernel(kernel.replace("_rope", "")), msa.set_attend_splits(splits)
+    old_r = msa.set_dec_rot_keys(0 if kernel == "dec_rope" else 256)
     try:
         c = _attend_case(rows=(1, 1, 2), n_loc=(65, 1, 9), n_mem=(0, 300, 61), q_start=(64, 0, 7), layer=23)
         g_out, g_f32, g_lse = _attend_gpu(msa, c, 16.0)
     finally:
+        msa.set_dec_rot_keys(old_r)
         msa.set_attend_splits(old_s)
         msa.set_attend_kernel(old_k)
     o_out, o_lse = oracle.attend(**c, pos_offset=16.0)

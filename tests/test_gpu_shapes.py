@@ -124,10 +124,14 @@ def test_gather_host_tier_head_counts(msa, hkv):
 
 # ----------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc", "tc_dec", "dec"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope"])
 def attend_kernel(request, msa):
-    old = msa.set_attend_kernel(request.param)
+    """dec: the decoding kernel rotating its local keys itself; dec_rope: the
+    same kernel after the separate rotation kernel."""
+    old = msa.set_attend_kernel(request.param.replace("_rope", ""))
+    old_r = msa.set_dec_rot_keys(0 if request.param == "dec_rope" else 256)
     yield request.param
+    msa.set_dec_rot_keys(old_r)
     msa.set_attend_kernel(old)
 
 
