@@ -49,6 +49,8 @@ def parse_args():
                    help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
+    p.add_argument("--topk-part", type=int, default=0,
+                   help="documents per CTA of the k <= 16 top-k (0: the library's plan)")
     p.add_argument("--dec-rot-keys", type=int, default=-1,
                    help="decoding attention: largest per-CTA share of local keys it rotates itself "
                         "(-1: the library's default; 0: always the separate rotation kernel)")
@@ -889,6 +891,8 @@ def config_of(w, eng, args, extra=None):
             cfg["attend_splits"] = args.attend_splits
         if args.dec_rot_keys >= 0:
             cfg["dec_rot_keys"] = args.dec_rot_keys
+        if args.topk_part:
+            cfg["topk_part"] = args.topk_part
     else:
         cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
     cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
@@ -953,6 +957,8 @@ def run_ours(args):
     msa.set_attend_splits(args.attend_splits)
     if args.dec_rot_keys >= 0:
         msa.set_dec_rot_keys(args.dec_rot_keys)
+    if args.topk_part:
+        msa.set_topk_part(args.topk_part)
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs

@@ -86,6 +86,7 @@ _sig("msa_debug_set_pf_pair", [ctypes.c_int])
 _sig("msa_debug_wait_probe", [ctypes.c_void_p])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_set_attend_splits", [ctypes.c_int])
+_sig("msa_debug_set_topk_part", [ctypes.c_int])
 _sig("msa_debug_set_dec_rot_keys", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
@@ -169,6 +170,13 @@ def set_attend_splits(n: int) -> int:
     the previous setting. Workspace sizes follow it: query attend_workspace
     after changing it. Benchmarking control."""
     return int(_lib.msa_debug_set_attend_splits(int(n)))
+
+
+def set_topk_part(n: int) -> int:
+    """Documents per CTA of the k <= 16 top-k (1024..16384, a power of two; 0:
+    the planned 2,048); returns the previous setting. Workspace sizes follow
+    it. Benchmarking control."""
+    return int(_lib.msa_debug_set_topk_part(int(n)))
 
 
 def set_dec_rot_keys(n: int) -> int:

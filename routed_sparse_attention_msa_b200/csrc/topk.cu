@@ -237,8 +237,13 @@ __global__ void __launch_bounds__(kWarps16 * 32) topk16_kernel(
   }
 }
 
+int g_topk_part = 0;  // testing control: documents per CTA of the k <= 16 path (0: kPartDocs)
+
+int part_docs() { return g_topk_part > 0 ? g_topk_part : kPartDocs; }
+
 int topk16_parts(int64_t n_docs) {
-  return n_docs <= kSinglePassDocs ? 1 : (int)((n_docs + kPartDocs - 1) / kPartDocs);
+  const int single = g_topk_part > 0 ? g_topk_part : kSinglePassDocs;
+  return n_docs <= single ? 1 : (int)((n_docs + part_docs() - 1) / part_docs());
 }
 
 // Generic path: one CTA (1024 threads) per sequence.
@@ -423,7 +428,7 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
       tickets = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(ws) +
                                             align_up((size_t)n_seq * parts * 16 * sizeof(uint64_t), 256));
       const dim3 grid((unsigned)parts, (unsigned)n_seq);
-      const int64_t per_cta = parts == 1 ? n_docs : kPartDocs;  // documents one CTA covers
+      const int64_t per_cta = parts == 1 ? n_docs : part_docs();  // documents one CTA covers
       const int it = per_cta <= 1024 ? 1 : per_cta <= 2048 ? 2 : per_cta <= 4096 ? 4 : per_cta <= 8192 ? 8 : 16;
       auto go = [&](auto kernel) {
         return launch_pdl(kernel, grid, dim3(kWarps16 * 32), 0, st, doc_key, n_docs, k, cand, tickets, top_ids,
@@ -459,3 +464,14 @@ msa_status launch_topk(const uint32_t* doc_key, int n_seq, int64_t n_docs, int k
 }
 
 }  // namespace msa
+
+// Documents per CTA of the k <= 16 top-k in later msa_route calls (1024..16384,
+// a power of two: 1,024 per batch of the CTA's 32 warps; 0 restores the
+// planned 2,048); returns the previous
+// setting. Workspace sizes follow it. A benchmarking control; not declared in
+// msa.h.
+extern "C" int msa_debug_set_topk_part(int n) {
+  const int old = msa::g_topk_part;
+  if (n == 0 || (n >= 1024 && n <= 16384 && (n & (n - 1)) == 0)) msa::g_topk_part = n;
+  return old;
+}
