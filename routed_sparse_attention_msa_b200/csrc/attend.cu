@@ -828,7 +828,10 @@ Layout layout(const msa_attend_args& a, const Shape& sh) {
   };
   if (sh.dec) {
     // the decoding kernel: the local keys rotated by rope_rows (bf16 high and low halves, 512 B)
-    if (!sh.rot) L.krot = take((size_t)std::max(sh.n_loc, 1) * a.hkv * 2 * kHeadDim * 2);
+    if (!sh.rot) {
+      L.qrot = take((size_t)a.n_q * a.hq * kHeadDim * 4);
+      L.krot = take((size_t)std::max(sh.n_loc, 1) * a.hkv * 2 * kHeadDim * 2);
+    }
   } else {
     L.qrot = take((size_t)a.n_q * a.hq * kHeadDim * 4);
     L.krot = take((size_t)(sh.n_loc > 0 ? sh.n_loc : 1) * a.hkv * kHeadDim * 4);
@@ -875,7 +878,7 @@ void fill_params(const msa_attend_args& a, const Shape& sh, const Layout& L, cha
     P.sel_chunk = reinterpret_cast<const int64_t*>(w + L.list_chunk);
   }
   P.rot_in_kernel = sh.rot ? 1 : 0;
-  P.rope_q = sh.dec ? 0 : 1;
+  P.rope_q = sh.dec && sh.rot ? 0 : 1;
   P.qrot = reinterpret_cast<float*>(w + L.qrot);
   P.krot = reinterpret_cast<float*>(w + L.krot);
   P.part_o = reinterpret_cast<float*>(w + L.part_o);
@@ -941,7 +944,7 @@ msa_status launch_attend(const msa_attend_args& a, void* ws, cudaStream_t st) {
     if (s != MSA_OK) return s;
   }
   if (sh.dec && sh.rot) return launch_attend_dec(P, st);  // rotates its own queries and local keys
-  if (sh.dec) {  // rope_rows rotates the local keys, the kernel its queries
+  if (sh.dec) {  // rope_rows rotates the queries and local keys
     s = launch_rope(P, a, sh, st);
     return s != MSA_OK ? s : launch_attend_dec(P, st);
   }

@@ -14,13 +14,14 @@
 //  - A CTA (one per SM) owns one kv head, one tile of query vectors and one
 //    split of the key list: an even share of the sequence's memory keys (the
 //    selected pooled rows) and of its local keys (the recent context).
-//  - The CTA rotates its own query vectors (global positions offset by k),
-//    and, when its share of the local keys is small, those keys too, as bf16
-//    high and low halves (so the logits keep fp32 accuracy) while the first
-//    memory rows are already in flight. Local steps come first, so those keys
-//    go straight into the shared-memory stages that will compute them. A
-//    larger share is rotated before the kernel by rope_rows (a kernel of its
-//    own that spreads the work over the whole GPU) and copied like the rest.
+//  - When its share of the local keys is small, the CTA rotates them
+//    (global positions offset by k) and its query vectors itself, as bf16
+//    high and low halves (so the logits keep fp32 accuracy), while the first
+//    memory rows are already in flight; local steps come first, so those keys
+//    go straight into the shared-memory stages that will compute them. With a
+//    larger share, rope_rows (a kernel of its own that spreads the work over
+//    the whole GPU) rotates the queries and local keys before the kernel, and
+//    the keys are copied like the rest.
 //    In the routed form the CTA lists the memory rows itself: the chunk
 //    ranges of the sequence's selected documents, scanned in shared memory.
 //  - Inside the CTA every warp is an independent flash-decoding worker: the
@@ -181,10 +182,16 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   if (tid < kHeadDim / 2) s_invf[tid] = p.inv_freq[tid];
   const int qv_v = tid >> 4, qv_d0 = 8 * (tid & 15);
   uint4 qraw = make_uint4(0, 0, 0, 0);
+  float4 qra = make_float4(0.f, 0.f, 0.f, 0.f), qrb = qra;  // rotated by rope_rows (rope_q)
   if (qv_v < nvec) {
     const int rr = qv_v / p.group, gg = qv_v - rr * p.group;
-    qraw = __ldcg(reinterpret_cast<const uint4*>(p.q + ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim +
-                                                 qv_d0));
+    const size_t qi = ((size_t)(row0 + rr) * p.hq + kvh * p.group + gg) * kHeadDim + qv_d0;
+    if (p.rope_q) {
+      qra = __ldcg(reinterpret_cast<const float4*>(p.qrot + qi));
+      qrb = __ldcg(reinterpret_cast<const float4*>(p.qrot + qi + 4));
+    } else {
+      qraw = __ldcg(reinterpret_cast<const uint4*>(p.q + qi));
+    }
   }
   const int nrot = p.rot_in_kernel ? (l1 - l0) * 32 : 0;  // at most 16 steps' keys (the host sees to it)
   auto kloc_ptr = [&](int it) {
@@ -300,7 +307,7 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     issue(w + kDWarps, r1, 1, p.rot_in_kernel);
   }
   int64_t r_next = row_of(w + 2 * kDWarps);  // row of key kl in the warp's third step
-  __syncthreads();  // the frequencies
+  if (!routed) __syncthreads();  // the frequencies (the routed listing's barriers cover them)
 
   // ---- rotate this CTA's local keys (global positions pos_offset + j) into bf16 high and low
   // halves, local step j straight into stage j / 8 of warp j % 8 (j < 16)
@@ -335,8 +342,8 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     uint32_t mine[4] = {qraw.x, qraw.y, qraw.z, qraw.w}, other[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) other[e] = __shfl_xor_sync(0xffffffffu, mine[e], 8);
-    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (qv_v < nvec) {
+    float y[8] = {qra.x, qra.y, qra.z, qra.w, qrb.x, qrb.y, qrb.z, qrb.w};
+    if (!p.rope_q && qv_v < nvec) {
       const double pos = p.pos_offset + (double)(g0 + qv_v / p.group);
       const bool first = qv_d0 < 64;  // this thread holds x0 (dims < 64) or x1 (dims >= 64) of its pairs
 #pragma unroll

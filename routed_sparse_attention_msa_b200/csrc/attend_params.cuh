@@ -20,7 +20,7 @@ struct AttnParams {
   int64_t n_docs, max_sel;
   int top_k;
   int rot_in_kernel;  // decoding kernel: 1 = it rotates its local keys itself, 0 = rope_rows did
-  int rope_q;         // rope_rows: 1 = rotate the query rows too (0: the decoding kernel does)
+  int rope_q;         // 1: rope_rows rotates the query rows (0: the decoding kernel does)
   float* qrot;      // [n_q, hq, d]
   float* krot;      // [n_loc, hkv, d], or [n_loc, hkv] rows of 512 B with krot_split
   float* part_o;    // [n_q, hq, splits, d]
@@ -73,10 +73,10 @@ msa_status launch_attend_dec_tc(const AttnParams& P, cudaStream_t st);
 // attend_dec.cu: the decoding shapes (at most 16 query vectors per tile),
 // grid (n_splits, hkv, n_tiles), each split an even share of every
 // sequence's memory and local keys; the splits of a (tile, kv head) form one
-// cluster. It rotates its own queries, and its local keys too when each
-// CTA's share is at most kDecRotKeys (otherwise rope_rows rotates them first,
-// krot_split = 1, rope_q = 0); it lists the routed form's memory rows itself
-// when top_k <= kDecRoutedMaxK.
+// cluster. It rotates its own queries and local keys when each CTA's share of
+// the local keys is small (otherwise rope_rows rotates both first, with
+// krot_split = 1); it lists the routed form's memory rows itself when
+// top_k <= kDecRoutedMaxK.
 constexpr int kDecMaxSplits = 8;
 constexpr int kDecRoutedMaxK = 256;
 constexpr int kDecRotKeysMax = 256;  // in-kernel rotation: the local keys of a CTA's first 16 steps at most
