@@ -87,6 +87,7 @@ _sig("msa_debug_wait_probe", [ctypes.c_void_p])
 _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_set_attend_splits", [ctypes.c_int])
 _sig("msa_debug_set_topk_part", [ctypes.c_int])
+_sig("msa_debug_set_tc_split_blocks", [ctypes.c_int])
 _sig("msa_debug_set_dec_rot_keys", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
@@ -170,6 +171,12 @@ def set_attend_splits(n: int) -> int:
     the previous setting. Workspace sizes follow it: query attend_workspace
     after changing it. Benchmarking control."""
     return int(_lib.msa_debug_set_attend_splits(int(n)))
+
+
+def set_tc_split_blocks(n: int) -> int:
+    """Fewest 64-key blocks per key split of the many-row tensor-core attention
+    (1..64); returns the previous setting. Benchmarking control."""
+    return int(_lib.msa_debug_set_tc_split_blocks(int(n)))
 
 
 def set_topk_part(n: int) -> int:

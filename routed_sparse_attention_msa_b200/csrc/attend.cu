@@ -714,7 +714,7 @@ struct Shape {
   bool rot;   // decoding kernel: it rotates its own local keys (rope_rows does otherwise)
   bool tc;    // tensor-core kernel (many rows per sequence)
   bool dec;   // decoding kernel (attend_dec.cu)
-  bool list;  // routed form listed into the workspace first (every kernel but the decoding one)
+  bool list;  // routed form listed into the workspace first (the split-K kernels, or top_k > 256)
 };
 
 // 0 automatic, 1 split-K, 2 tensor cores, 3 decoding tensor cores, 4 decoding
@@ -722,6 +722,7 @@ struct Shape {
 int g_attend_kernel = 0;
 int g_attend_splits = 0;  // forward split-K key splits: 0 = planned below, else forced (testing control)
 int g_dec_rot_keys = 48;  // decoding kernel: largest local-key share per CTA it rotates itself
+int g_tc_split_blocks = 2;  // tensor-core kernel: fewest 64-key blocks per key split
 
 // allow_tc: the forward may take the tensor-core kernel when the query
 // vectors of a sequence fill at least half of its 128-vector tile.
@@ -746,16 +747,16 @@ Shape plan_kernel(const msa_attend_args& a, bool allow_tc) {
     }
     sh.n_loc = a.loc_off[a.n_seq];
     // split the 64-key blocks across CTAs while (tiles x kv heads) is under one
-    // wave, keeping at least 4 blocks per split: a CTA pipelines its blocks
-    // (the next one's copies and S overlap the current one's softmax), while a
-    // split pays a partial write and a merge (1M prefill, 4 blocks per tile:
-    // 4 splits 73.9 us per layer, 1 split 55.0 us)
+    // wave, keeping at least g_tc_split_blocks blocks per split: a CTA pipelines
+    // its blocks (the next one's copies and S overlap the current one's
+    // softmax), a split pays the cluster's merge; the splits of a (tile, kv
+    // head) are one cluster, so at most 8
     const int64_t ctas = (int64_t)sh.n_tiles * a.hkv;
     const int64_t blocks = (a.max_sel + max_loc + 63) / 64;
     int64_t splits = ctas > 0 ? (148 + ctas - 1) / ctas : 1;
-    splits = std::min<int64_t>(splits, (blocks + 3) / 4);
+    splits = std::min<int64_t>(splits, (blocks + g_tc_split_blocks - 1) / g_tc_split_blocks);
     if (g_attend_splits > 0) splits = g_attend_splits;  // testing control
-    splits = std::min<int64_t>(std::min<int64_t>(splits, blocks), 64);
+    splits = std::min<int64_t>(std::min<int64_t>(splits, blocks), 8);
     sh.n_splits = (int)std::max<int64_t>(splits, 1);
     return sh;
   }
@@ -810,7 +811,8 @@ Shape plan_kernel(const msa_attend_args& a, bool allow_tc) {
 
 Shape plan(const msa_attend_args& a, bool allow_tc) {
   Shape sh = plan_kernel(a, allow_tc);
-  sh.list = a.sel_off == nullptr && !(sh.dec && a.top_k <= kDecRoutedMaxK);
+  // the decoding and tensor-core kernels list the routed form's rows themselves
+  sh.list = a.sel_off == nullptr && !((sh.dec || sh.tc) && a.top_k <= kDecRoutedMaxK);
   return sh;
 }
 
@@ -1034,5 +1036,14 @@ extern "C" int msa_debug_set_attend_splits(int n) {
 extern "C" int msa_debug_set_dec_rot_keys(int n) {
   const int old = msa::g_dec_rot_keys;
   if (n >= 0 && n <= msa::kDecRotKeysMax) msa::g_dec_rot_keys = n;
+  return old;
+}
+
+// Fewest 64-key blocks per key split of the many-row tensor-core attention in
+// later msa_attend calls (1..64); returns the previous setting. Workspace
+// sizes follow it. A benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_tc_split_blocks(int n) {
+  const int old = msa::g_tc_split_blocks;
+  if (n >= 1 && n <= 64) msa::g_tc_split_blocks = n;
   return old;
 }

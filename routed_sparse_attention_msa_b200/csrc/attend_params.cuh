@@ -59,8 +59,9 @@ __device__ __forceinline__ int seq_of(const int32_t* off, int n_seq, int x) {
 }
 
 // attend_tc.cu: one CTA per (tile of 128 query vectors = rt rows x group q
-// heads, kv head); grid (n_tiles, hkv). Needs rope_rows to have run with
-// krot_split = 1.
+// heads, kv head, key split); grid (n_tiles, hkv, n_splits), the splits of a
+// (tile, kv head) one cluster. Needs rope_rows to have run with krot_split =
+// 1; lists the routed form's memory rows itself when top_k <= kDecRoutedMaxK.
 constexpr int kAttnTcVec = 128;
 msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st);
 int attend_tc_error_take();  // 1 if its bounded wait ran out since the last call

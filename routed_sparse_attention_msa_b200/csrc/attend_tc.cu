@@ -21,8 +21,10 @@
 //                 when the running max passes it by more than 2^11.5; then
 //                 the two threads rescale their halves of the O row in TMEM).
 // When (tiles x kv heads) would not fill the GPU, the key blocks are split
-// across CTAs, each writing an unnormalised partial that the last one to
-// finish merges by log-sum-exp.
+// across CTAs: the splits of a (tile, kv head), at most 8, are one
+// thread-block cluster; each leaves its unnormalised partial (o, m, l) in its
+// shared memory and the cluster's CTAs share out the query vectors and merge
+// the splits by log-sum-exp straight from each other's shared memory.
 // The rotated queries and local keys are split into a bf16 high part and the
 // bf16 rounding of the remainder (the local keys by rope_rows), and S sums
 // Qhi Khi + Qlo Khi + Qhi Klo (the Qlo Klo term is below 2^-16 of the
@@ -68,6 +70,9 @@ static_assert(kStageTc % 1024 == 0 && offStage % 1024 == 0 && offVT % 1024 == 0 
               "128-byte-swizzle atoms start on 1024-byte boundaries");
 static_assert(kSmemTc <= 227 * 1024, "shared memory per CTA");
 constexpr int kTmemCols = 256;  // S: columns 0..63, O block: 128..255
+constexpr int kMaxClusterTc = 8;  // key splits per (tile, kv head): one portable cluster
+constexpr int kPO = kHeadDim + 4;  // row stride (floats) of a CTA's partial output in shared memory
+static_assert(kVec * (kPO + 2) * 4 <= 2 * kStageTc, "the partial fits the stages");
 // instruction descriptors: D fp32, A/B bf16, K-major; M = 128; N = 64 or 128
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNK >> 3) << 17) | (8u << 24);
 constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) | (8u << 24);
@@ -83,6 +88,33 @@ template <int N>
 __device__ __forceinline__ void cp_wait_tc() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float bf_round(float x) { return __uint_as_float(f2bf_bits(x) << 16); }
+
+// ---- thread-block cluster: the key splits of one (tile, kv head)
+__device__ __forceinline__ uint32_t cluster_rank_tc() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_tc() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float ld_cluster(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a) : "memory");
+  return v;
+}
 
 // Eight fp32 values -> 16-byte bf16 high part and 16-byte bf16 remainder.
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
@@ -135,8 +167,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   }
   pdl_wait();  // the rotated rows and the selection come from earlier kernels
   pdl_trigger();
-  const int64_t mem_base = __ldg(p.sel_off + s);
-  const int64_t n_mem = __ldg(p.sel_off + s + 1) - mem_base;
+  // the sequence's memory rows: the gather listing, or in the routed form the chunks of its
+  // selected documents in rank order (their first list positions scanned in shared memory)
+  __shared__ int64_t s_pre[kDecRoutedMaxK + 1], s_c0[kDecRoutedMaxK], s_wsum[kThreadsTc / 32];
+  const bool routed = p.sel_off == nullptr;
+  int64_t mem_base = 0, n_mem;
+  if (routed) {
+    int64_t c0 = 0, cnt = 0;
+    if (tid < p.top_k) {
+      const int32_t doc = __ldcg(p.top_ids + (size_t)s * p.top_k + tid);
+      if (doc >= 0 && doc < p.n_docs) {
+        c0 = __ldcg(p.doc_chunk_off + doc);
+        cnt = __ldcg(p.doc_chunk_off + doc + 1) - c0;
+      }
+    }
+    int64_t x = cnt;  // inclusive scan over the block (top_k <= 256 = its threads)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wsum[warp] = x;
+    __syncthreads();
+    for (int j = 0; j < warp; ++j) x += s_wsum[j];
+    if (tid < p.top_k) {
+      s_pre[tid] = x - cnt;
+      s_c0[tid] = c0;
+    }
+    if (tid == p.top_k - 1) s_pre[p.top_k] = x;
+    __syncthreads();
+    n_mem = min(s_pre[p.top_k], p.max_sel);
+  } else {
+    mem_base = __ldg(p.sel_off + s);
+    n_mem = __ldg(p.sel_off + s + 1) - mem_base;
+  }
   const int64_t n_keys = n_mem + lvis;
   // this CTA's share of the key blocks (split-K when the grid is small)
   const int64_t n_blocks = (n_keys + kNK - 1) / kNK;
@@ -151,7 +215,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   auto load_idx = [&](int b, int j) -> int64_t {
     const int64_t key = k_begin + (int64_t)b * kNK + j;
     if (b >= nblk || key >= k_end || key >= n_mem) return -1;
-    return p.sel_chunk ? __ldcg(p.sel_chunk + mem_base + key) : mem_base + key;
+    if (!routed) return p.sel_chunk ? __ldcg(p.sel_chunk + mem_base + key) : mem_base + key;
+    int lo = 0, hi = p.top_k - 1;  // the last document whose first list position is <= key
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= key) lo = mid; else hi = mid - 1;
+    }
+    return s_c0[lo] + (key - s_pre[lo]);
   };
   auto issue = [&](int b) {
     if (b < nblk) {
@@ -388,61 +458,69 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
   const size_t rh = (size_t)row * p.hq + h;
 
   if (p.n_splits > 1) {
-    // ---- split-K: unnormalised partial (o, m, l) out; the last CTA of the
-    // (tile, kv head) merges by log-sum-exp
-    __shared__ int s_last;
-    const size_t pi = rh * p.n_splits + sp_idx;
-    if (ok) {
+    // ---- split-K inside the cluster: this CTA's unnormalised partial (o, m, l) goes to its
+    // shared memory (the stages, idle now); after the barrier CTA r merges the vectors v with
+    // v % splits == r from every CTA's memory, and the second barrier keeps that memory alive
+    float* po = reinterpret_cast<float*>(smem + offStage);  // [128 vectors][kPO]
+    float* pm = po + kVec * kPO;                            // [128]
+    float* pl = pm + kVec;                                  // [128]
+    const bool have = ok && blk > 0;  // uniform: every thread of the CTA walked the same blocks
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        float t[16];
-        if (blk > 0) {
-          tmem_ld16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
-          tmem_ld_wait();
-        } else {
+    for (int cc = 0; cc < 4; ++cc) {
+      float t[16];
+      if (have) {
+        tmem_ld16(tmem_o + lane_base + 64 * hs + 16 * cc, t);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) t[j] = 0.f;
-        }
-        if (vvalid) {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + pi * kHeadDim + 64 * hs + 16 * cc);
-          dst[0] = make_float4(t[0], t[1], t[2], t[3]);
-          dst[1] = make_float4(t[4], t[5], t[6], t[7]);
-          dst[2] = make_float4(t[8], t[9], t[10], t[11]);
-          dst[3] = make_float4(t[12], t[13], t[14], t[15]);
-        }
+        for (int j = 0; j < 16; ++j) t[j] = 0.f;
       }
-      if (vvalid && hs == 0) p.part_ml[pi] = make_float2(m_ref, l);
+      float4* dst = reinterpret_cast<float4*>(po + v * kPO + 64 * hs + 16 * cc);
+      dst[0] = make_float4(t[0], t[1], t[2], t[3]);
+      dst[1] = make_float4(t[4], t[5], t[6], t[7]);
+      dst[2] = make_float4(t[8], t[9], t[10], t[11]);
+      dst[3] = make_float4(t[12], t[13], t[14], t[15]);
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.tickets + (size_t)tile * p.hkv + kvh, 1u) == (unsigned)(p.n_splits - 1);
-    __syncthreads();
-    if (s_last && vvalid) {
-      __threadfence();
-      float mm = -INFINITY;
-      for (int j = 0; j < p.n_splits; ++j) {
-        const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
-        if (x.y > 0.f) mm = fmaxf(mm, x.x);
+    if (hs == 0) {
+      pm[v] = m_ref;
+      pl[v] = have ? l : 0.f;
+    }
+    cluster_sync_tc();
+    const int ns = p.n_splits;
+    if (vvalid && v % ns == (int)cluster_rank_tc()) {
+      float mj[kMaxClusterTc], lj[kMaxClusterTc];
+#pragma unroll
+      for (int j = 0; j < kMaxClusterTc; ++j) {
+        lj[j] = 0.f;
+        mj[j] = -INFINITY;
+        if (j < ns) {
+          lj[j] = ld_cluster(cluster_addr(pl + v, j));
+          mj[j] = ld_cluster(cluster_addr(pm + v, j));
+        }
       }
-      float wsum = 0.f;
-      for (int j = 0; j < p.n_splits; ++j) {
-        const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
-        if (x.y > 0.f) wsum += x.y * exp2f(x.x - mm);
+      float mm = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMaxClusterTc; ++j)
+        if (lj[j] > 0.f) mm = fmaxf(mm, mj[j]);
+      float wj[kMaxClusterTc], wsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxClusterTc; ++j) {
+        wj[j] = lj[j] > 0.f ? exp2f(mj[j] - mm) : 0.f;
+        wsum += lj[j] * wj[j];
       }
       const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
       const size_t base = rh * kHeadDim + 64 * hs;
-#pragma unroll 4  // several dimension chunks' loads in flight
+#pragma unroll 1
       for (int d = 0; d < 64; d += 8) {
         float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < p.n_splits; ++j) {
-          const float2 x = __ldcg(p.part_ml + rh * p.n_splits + j);
-          if (!(x.y > 0.f)) continue;
-          const float w = exp2f(x.x - mm);
-          const float4* src =
-              reinterpret_cast<const float4*>(p.part_o + (rh * p.n_splits + j) * kHeadDim + 64 * hs + d);
-          const float4 a = __ldcg(src), b = __ldcg(src + 1);
-          r[0] += w * a.x; r[1] += w * a.y; r[2] += w * a.z; r[3] += w * a.w;
-          r[4] += w * b.x; r[5] += w * b.y; r[6] += w * b.z; r[7] += w * b.w;
+#pragma unroll
+        for (int j = 0; j < kMaxClusterTc; ++j) {
+          if (wj[j] > 0.f) {
+            const uint32_t a = cluster_addr(po + v * kPO + 64 * hs + d, j);
+            const float4 x = ld_cluster4(a), y = ld_cluster4(a + 16);
+            r[0] += wj[j] * x.x; r[1] += wj[j] * x.y; r[2] += wj[j] * x.z; r[3] += wj[j] * x.w;
+            r[4] += wj[j] * y.x; r[5] += wj[j] * y.y; r[6] += wj[j] * y.z; r[7] += wj[j] * y.w;
+          }
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) r[i] *= inv;
@@ -455,6 +533,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attend_tc_kernel(const __grid_c
       }
       if (p.lse && hs == 0) p.lse[rh] = wsum > 0.f ? (mm + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
     }
+    cluster_sync_tc();
   } else if (ok) {  // ---- one CTA per (tile, kv head): normalised output, log-sum-exp
     const float inv = l > 0.f ? 1.0f / l : 0.f;
     const size_t base = rh * kHeadDim + 64 * hs;
@@ -501,9 +580,21 @@ msa_status launch_attend_tc(const AttnParams& P, cudaStream_t st) {
   static std::atomic<uint64_t> attr{0};
   cudaError_t e = smem_limit_once(attend_tc_kernel, kSmemTc, attr);
   if (e != cudaSuccess) return cuda_fail(e, "attend: tensor-core kernel shared memory");
-  e = launch_pdl(attend_tc_kernel, dim3((unsigned)P.n_tiles, (unsigned)P.hkv, (unsigned)P.n_splits),
-                             dim3(kThreadsTc),
-                             (size_t)kSmemTc, st, P);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P.n_tiles, (unsigned)P.hkv, (unsigned)P.n_splits);
+  cfg.blockDim = dim3(kThreadsTc);
+  cfg.dynamicSmemBytes = (size_t)kSmemTc;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;  // the key splits of a (tile, kv head): one cluster
+  at[1].val.clusterDim.x = 1;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = (unsigned)P.n_splits;
+  cfg.attrs = at;
+  cfg.numAttrs = P.n_splits > 1 ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: tensor cores (many rows)");
   return launch_check("attend: tensor cores (many rows)");
 }

@@ -87,7 +87,17 @@ def check_prefill_attention(msa, bank, ids, w, layer, seqs):
     lse = torch.empty((S * R, w.hq), dtype=torch.float32, device="cuda")
     ws = torch.empty(msa.attend_workspace(*args, pos_offset=float(w.top_k)), dtype=torch.uint8, device="cuda")
     msa.attend(*args, out, ws, out_f32=of, lse=lse, pos_offset=float(w.top_k))
+    # the routed form (what bench.py runs for content in HBM): identical results
+    routed = (top_d, bank.layer_c.doc_chunk_off)
+    r_args = args[:8] + (None, None, cap)
+    r_out, r_of = torch.empty_like(out), torch.empty_like(of)
+    r_lse = torch.empty_like(lse)
+    r_ws = torch.empty(msa.attend_workspace(*r_args, pos_offset=float(w.top_k), routed=routed), dtype=torch.uint8,
+                       device="cuda")
+    msa.attend(*r_args, r_out, r_ws, out_f32=r_of, lse=r_lse, pos_offset=float(w.top_k), routed=routed)
     msa.sync_check()
+    np.testing.assert_array_equal(bits(r_out), bits(out))
+    np.testing.assert_array_equal(r_of.cpu().numpy(), of.cpu().numpy())
     of, lse = of.cpu().numpy(), lse.cpu().numpy()
     so = sel_off.cpu().numpy()
     sc = sel.cpu().numpy()
@@ -103,6 +113,33 @@ def check_prefill_attention(msa, bank, ids, w, layer, seqs):
                                      pos_offset=float(w.top_k))
         assert np.abs(of[r] - o_out).max() <= 1e-2, s_
         np.testing.assert_allclose(lse[r], o_lse, atol=1e-3, rtol=0)
+
+
+def check_decode_attention_routed(msa, bank, ids, w, layer, n_loc):
+    """One decoding row per sequence in the routed form (attention lists the
+    selected chunks from the route's ids), in bench.py's launch configuration,
+    against the oracle chain (oracle.gather, oracle.attend)."""
+    S = ids.shape[0]
+    q = host_normal((S, w.hq, 128), synth.tid("q_att", layer, 2))
+    kl = host_normal((S * n_loc, w.hkv, 128), synth.tid("k_loc", layer, 2))
+    vl = host_normal((S * n_loc, w.hkv, 128), synth.tid("v_loc", layer, 2))
+    qso, qst, lo = np.arange(S + 1), np.full(S, n_loc - 1), np.arange(S + 1) * n_loc
+    cap = w.top_k * bank.layer_c.max_doc_chunks
+    routed = (torch.from_numpy(ids).cuda(), bank.layer_c.doc_chunk_off)
+    args = (from_bits(q), qso, qst, from_bits(kl), from_bits(vl), lo, bank.kbar, bank.vbar, None, None, cap)
+    out = torch.empty((S, w.hq, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((S, w.hq, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((S, w.hq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(msa.attend_workspace(*args, pos_offset=float(w.top_k), routed=routed), dtype=torch.uint8,
+                     device="cuda")
+    msa.attend(*args, out, ws, out_f32=of, lse=lse, pos_offset=float(w.top_k), routed=routed)
+    msa.sync_check()
+    o_off, o_sel = oracle.gather(ids, bank.dco)
+    kh, vh = bank.host_content()
+    o_out, o_lse = oracle.attend(q, qso, qst, kl, vl, lo, kh, vh, o_off, o_sel, pos_offset=float(w.top_k))
+    assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+    np.testing.assert_allclose(lse.cpu().numpy(), o_lse, atol=1e-3, rtol=0)
+    np.testing.assert_array_equal(bits(out), synth.bf16_bits(of.cpu().numpy()))
 
 
 # ------------------------------------------------------------------ tiny
@@ -143,6 +180,9 @@ def test_1m_decode_all_layers_and_prefill(msa):
             assert set(pid[0].tolist()) == set(planp.docs[0])
             # its attention (128 rows over 16 documents + 128 causal local keys), full oracle
             check_prefill_attention(msa, bank, pid, w, layer, seqs=[0])
+            # a decoding step of the same layer in the routed form (one row after 129 local
+            # keys: five key splits in one cluster per kv head, local keys rotated in the kernel)
+            check_decode_attention_routed(msa, bank, ids, w, layer, n_loc=129)
         del bank
     assert n_exact >= w.n_layers - 1  # rank-k gap >= 1e-2 on (almost) every layer
 
@@ -189,6 +229,8 @@ def test_10m_prefill_and_decode_sampled(msa):
     kh, vh = bank.host_content()
     o_out, _ = oracle.attend(q, qso_a, qst, kl, vl, lo, kh, vh, o_off, o_sel, pos_offset=float(w.top_k))
     assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+    # the same step in the routed form, as bench.py runs it
+    check_decode_attention_routed(msa, bank, ids, w, 0, n_loc=L)
 
 
 # ------------------------------------------------------------------ 100m

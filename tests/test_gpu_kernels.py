@@ -480,6 +480,25 @@ def test_attend_forced_splits(msa, kernel, splits):
     np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
 
 
+@pytest.mark.parametrize("splits", [1, 2, 3, 8])
+def test_attend_tc_cluster_splits(msa, splits):
+    """The many-row tensor-core attention with its key blocks split over a
+    cluster of 1 to 8 CTAs (merged from each other's shared memory): a
+    sequence with 9 key blocks, one with 2 (splits beyond its blocks get
+    none), prefill rows after a local prefix."""
+    old_k, old_s = msa.set_attend_kernel("tc"), msa.set_attend_splits(splits)
+    try:
+        c = _attend_case(rows=(64, 40), n_loc=(64, 70), n_mem=(500, 60), q_start=(0, 30), layer=24)
+        g_out, g_f32, g_lse = _attend_gpu(msa, c, 16.0)
+    finally:
+        msa.set_attend_splits(old_s)
+        msa.set_attend_kernel(old_k)
+    o_out, o_lse = oracle.attend(**c, pos_offset=16.0)
+    assert np.abs(g_f32 - o_out).max() <= 1e-2
+    np.testing.assert_array_equal(g_out, synth.bf16_bits(g_f32))
+    np.testing.assert_allclose(g_lse, o_lse, atol=1e-3, rtol=0)
+
+
 # ------------------------------------------------------- whole step, tiny
 
 def test_tiny_step_route_gather_attend(msa):
