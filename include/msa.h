@@ -172,7 +172,9 @@ msa_status msa_bank_norms(const uint16_t* kbar_r, int64_t n_chunks, int32_t hr, 
  * order of decreasing score, equal scores by increasing document id:
  * top_ids [n_seq, k] int32 and top_scores [n_seq, k] fp32 (device).
  * all_doc_scores (device [n_seq, n_docs] fp32, or NULL) receives every score.
- * Limits: d = 128, n_seq <= 256, top_k <= 4096.
+ * Limits: d = 128, top_k <= 4096. More than 256 sequences run as successive
+ * groups of 256 on `stream` (each group streams the bank once); the
+ * workspace is sized for one group.
  * How it runs (not part of the contract): with hr = 8 and up to 64 rows in a
  * call the scorer streams the bank once with all heads' accumulators in
  * tensor memory (bound by HBM bandwidth); above 64 rows it contracts the
@@ -317,7 +319,9 @@ msa_status msa_gather(const msa_gather_args* args, void* stream);
  * attend; msa_attend_backward does not take it (MSA_ERR_UNSUPPORTED).
  * out is bf16 (nearest even of the fp32 result); out_f32 and lse are optional.
  * max_sel >= sel_off[s+1] - sel_off[s] for every s sizes the split-K grid.
- * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16, n_seq <= 256. q, k_loc,
+ * Limits: d = 128, hq % hkv == 0, hq / hkv <= 16. More than 256 sequences
+ * run as successive groups of 256 on `stream` with one workspace (sized for
+ * the largest group); msa_attend_backward takes at most 256. q, k_loc,
  * v_loc, mem_k, mem_v, out and out_f32 must be 16-byte aligned and the
  * workspace 256-byte aligned (MSA_ERR_INVALID_ARG / MSA_ERR_WORKSPACE).
  * How it runs (not part of the contract): when a sequence's query vectors

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <thread>
@@ -199,36 +200,24 @@ msa_status msa_route_workspace(const msa_bank_layer* b, int32_t n_seq, int32_t n
                                size_t* bytes) {
   msa_status s = check_bank(b, false);
   if (s != MSA_OK) return s;
-  if (!bytes || n_seq <= 0 || n_seq > kMaxSeq || n_rows < n_seq || top_k <= 0)
+  if (!bytes || n_seq <= 0 || n_rows < n_seq || top_k <= 0)
     return fail(MSA_ERR_INVALID_ARG, "route_workspace: bad sizes");
   if ((top_k < b->n_docs ? top_k : b->n_docs) > 4096)
     return fail(MSA_ERR_UNSUPPORTED, "route_workspace: min(top_k, n_docs) > 4096");
-  *bytes = route_layout(b, n_seq, n_rows, top_k).total;
+  *bytes = route_layout(b, n_seq < kMaxSeq ? n_seq : kMaxSeq, n_rows, top_k).total;
   return MSA_OK;
 }
 
-msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t* q_seq_off, int32_t n_seq,
-                     int32_t n_rows, int32_t top_k, float eps, int32_t* top_ids, float* top_scores,
-                     float* all_doc_scores, void* ws, size_t ws_bytes, void* stream) {
-  msa_status s = check_bank(b, false);
-  if (s != MSA_OK) return s;
-  if (n_seq <= 0 || n_seq > kMaxSeq) return fail(MSA_ERR_UNSUPPORTED, "route: n_seq = %d (1..%d)", n_seq, kMaxSeq);
-  if (top_k <= 0) return fail(MSA_ERR_INVALID_ARG, "route: top_k = %d", top_k);
-  if ((top_k < b->n_docs ? top_k : b->n_docs) > 4096)
-    return fail(MSA_ERR_UNSUPPORTED, "route: min(top_k, n_docs) = %lld > 4096",
-                (long long)(top_k < b->n_docs ? top_k : b->n_docs));
-  if (!qr || !q_seq_off || !top_ids || !top_scores) return fail(MSA_ERR_INVALID_ARG, "route: NULL pointer");
-  if (!(eps > 0.f)) return fail(MSA_ERR_INVALID_ARG, "route: eps must be > 0");
-  if (q_seq_off[0] != 0 || q_seq_off[n_seq] != n_rows)
-    return fail(MSA_ERR_INVALID_ARG, "route: q_seq_off must start at 0 and end at n_rows");
-  for (int i = 0; i < n_seq; ++i)
-    if (q_seq_off[i + 1] <= q_seq_off[i])
-      return fail(MSA_ERR_INVALID_ARG, "route: sequence %d has no query rows", i);
-  RouteLayout L = route_layout(b, n_seq, n_rows, top_k);
-  if (!ws || ws_bytes < L.total)
-    return fail(MSA_ERR_WORKSPACE, "route: workspace %zu B, need %zu B", ws_bytes, L.total);
-  cudaStream_t st = (cudaStream_t)stream;
-  char* w = reinterpret_cast<char*>(ws);
+namespace msa {
+namespace {
+
+// The routing kernels over one group of at most kMaxSeq sequences: q_seq_off
+// rebased to the group's first row, outputs already offset to its first
+// sequence; the workspace is laid out for kMaxSeq sequences (or fewer) and
+// the call's whole row count, so every group fits it.
+msa_status route_group(const msa_bank_layer* b, const uint16_t* qr, const int32_t* q_seq_off, int n_seq, int n_rows,
+                       int top_k, float eps, int32_t* top_ids, float* top_scores, float* all_doc_scores, char* w,
+                       const RouteLayout& L, cudaStream_t st) {
   RoutePlan p;
   p.qr = qr; p.kr_inv_norm = b->kr_inv_norm; p.chunk_doc = b->chunk_doc; p.kbar_r = b->kbar_r;
   p.n_chunks = b->n_chunks; p.n_docs = b->n_docs; p.hr = b->hr; p.n_rows = n_rows; p.n_seq = n_seq;
@@ -246,9 +235,7 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   int which = g_score_kernel;
   if (which == 0)
     which = score_pf_supported(p) && n_rows > kManyRows ? 3 : score_tc_supported(p) ? 2 : 1;
-  if (b->n_chunks > 0 && ((which == 2 && !score_tc_supported(p)) || (which == 3 && !score_pf_supported(p))))
-    return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
-  s = launch_qprep(p, eps, st);
+  msa_status s = launch_qprep(p, eps, st);
   if (s != MSA_OK) return s;
   if (b->n_chunks > 0) {
     record_debug_event(0, st);
@@ -258,6 +245,54 @@ msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t*
   }
   int k = top_k < b->n_docs ? top_k : (int)b->n_docs;
   return launch_topk(p.doc_key, n_seq, b->n_docs, k, top_ids, top_scores, all_doc_scores, w + L.topk, st);
+}
+
+}  // namespace
+}  // namespace msa
+
+msa_status msa_route(const msa_bank_layer* b, const uint16_t* qr, const int32_t* q_seq_off, int32_t n_seq,
+                     int32_t n_rows, int32_t top_k, float eps, int32_t* top_ids, float* top_scores,
+                     float* all_doc_scores, void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_bank(b, false);
+  if (s != MSA_OK) return s;
+  if (n_seq <= 0) return fail(MSA_ERR_UNSUPPORTED, "route: n_seq = %d (1..)", n_seq);
+  if (top_k <= 0) return fail(MSA_ERR_INVALID_ARG, "route: top_k = %d", top_k);
+  if ((top_k < b->n_docs ? top_k : b->n_docs) > 4096)
+    return fail(MSA_ERR_UNSUPPORTED, "route: min(top_k, n_docs) = %lld > 4096",
+                (long long)(top_k < b->n_docs ? top_k : b->n_docs));
+  if (!qr || !q_seq_off || !top_ids || !top_scores) return fail(MSA_ERR_INVALID_ARG, "route: NULL pointer");
+  if (!(eps > 0.f)) return fail(MSA_ERR_INVALID_ARG, "route: eps must be > 0");
+  if (q_seq_off[0] != 0 || q_seq_off[n_seq] != n_rows)
+    return fail(MSA_ERR_INVALID_ARG, "route: q_seq_off must start at 0 and end at n_rows");
+  for (int i = 0; i < n_seq; ++i)
+    if (q_seq_off[i + 1] <= q_seq_off[i])
+      return fail(MSA_ERR_INVALID_ARG, "route: sequence %d has no query rows", i);
+  const int group = n_seq < kMaxSeq ? n_seq : kMaxSeq;
+  RouteLayout L = route_layout(b, group, n_rows, top_k);
+  if (!ws || ws_bytes < L.total)
+    return fail(MSA_ERR_WORKSPACE, "route: workspace %zu B, need %zu B", ws_bytes, L.total);
+  {
+    RoutePlan probe;
+    probe.qr = qr; probe.kbar_r = b->kbar_r; probe.hr = b->hr; probe.n_chunks = b->n_chunks;
+    const int which = g_score_kernel;
+    if (b->n_chunks > 0 && ((which == 2 && !score_tc_supported(probe)) || (which == 3 && !score_pf_supported(probe))))
+      return fail(MSA_ERR_UNSUPPORTED, "route: tensor-core scoring needs hr = 8");
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = reinterpret_cast<char*>(ws);
+  const int k = top_k < b->n_docs ? top_k : (int)b->n_docs;
+  // more than kMaxSeq sequences: one pass of the kernels per group of kMaxSeq, in order on the
+  // stream (each group streams the bank once)
+  int32_t qso[kMaxSeq + 1];
+  for (int s0 = 0; s0 < n_seq; s0 += kMaxSeq) {
+    const int gs = n_seq - s0 < kMaxSeq ? n_seq - s0 : kMaxSeq;
+    for (int i = 0; i <= gs; ++i) qso[i] = q_seq_off[s0 + i] - q_seq_off[s0];
+    s = route_group(b, qr + (size_t)q_seq_off[s0] * b->hr * kHeadDim, qso, gs, qso[gs], top_k, eps,
+                    top_ids + (size_t)s0 * k, top_scores + (size_t)s0 * k,
+                    all_doc_scores ? all_doc_scores + (size_t)s0 * b->n_docs : nullptr, w, L, st);
+    if (s != MSA_OK) return s;
+  }
+  return MSA_OK;
 }
 
 msa_status msa_topk_merge(const int32_t* ids, const float* scores, const int64_t* id_offset, int32_t n_shards,
@@ -280,7 +315,7 @@ msa_status msa_gather(const msa_gather_args* a, void* stream) {
   msa_status s = check_bank(a->bank, true);
   if (s != MSA_OK) return s;
   const msa_bank_layer& b = *a->bank;
-  if (a->n_seq <= 0 || a->n_seq > kMaxSeq || a->top_k <= 0) return fail(MSA_ERR_INVALID_ARG, "gather: bad sizes");
+  if (a->n_seq <= 0 || a->top_k <= 0) return fail(MSA_ERR_INVALID_ARG, "gather: bad sizes");
   if (!a->top_ids || !a->sel_off || !a->sel_chunk) return fail(MSA_ERR_INVALID_ARG, "gather: NULL pointer");
   const int k = a->top_k < b.n_docs ? a->top_k : (int)b.n_docs;
   const int64_t need = (int64_t)a->n_seq * k * b.max_doc_chunks;
@@ -360,7 +395,7 @@ static msa_status check_attend(const msa_attend_args* a) {
   if (a->hkv <= 0 || a->hq <= 0 || a->hq % a->hkv) return fail(MSA_ERR_INVALID_ARG, "attend: hq must be a multiple of hkv");
   const int g = a->hq / a->hkv;
   if (g > 16 || (g & (g - 1))) return fail(MSA_ERR_UNSUPPORTED, "attend: hq / hkv = %d (1, 2, 4, 8 or 16)", g);
-  if (a->n_seq <= 0 || a->n_seq > kMaxSeq) return fail(MSA_ERR_UNSUPPORTED, "attend: n_seq = %d (1..%d)", a->n_seq, kMaxSeq);
+  if (a->n_seq <= 0) return fail(MSA_ERR_UNSUPPORTED, "attend: n_seq = %d (1..)", a->n_seq);
   if (!a->q || !a->q_seq_off || !a->q_start || !a->loc_off || !a->out)
     return fail(MSA_ERR_INVALID_ARG, "attend: NULL pointer");
   if (!a->sel_off == !a->top_ids)
@@ -390,22 +425,79 @@ static msa_status check_attend(const msa_attend_args* a) {
   return MSA_OK;
 }
 
+namespace {
+
+// The sequences s0 .. s1 - 1 of an attention call (at most kMaxSeq) as a call
+// of their own: host offsets rebased, device row arrays and outputs offset to
+// the group's first row, local key and sequence.
+struct AttendGroup {
+  msa_attend_args a;
+  int32_t qso[kMaxSeq + 1], qst[kMaxSeq], lo[kMaxSeq + 1];
+};
+
+void attend_group(const msa_attend_args& a, int s0, int s1, AttendGroup& g) {
+  g.a = a;
+  const int row0 = a.q_seq_off[s0], loc0 = a.loc_off[s0], n = s1 - s0;
+  for (int i = 0; i <= n; ++i) {
+    g.qso[i] = a.q_seq_off[s0 + i] - row0;
+    g.lo[i] = a.loc_off[s0 + i] - loc0;
+    if (i < n) g.qst[i] = a.q_start[s0 + i];
+  }
+  const size_t qrow = (size_t)a.hq * kHeadDim, krow = (size_t)a.hkv * kHeadDim;
+  g.a.n_seq = n;
+  g.a.n_q = g.qso[n];
+  g.a.q_seq_off = g.qso;
+  g.a.q_start = g.qst;
+  g.a.loc_off = g.lo;
+  g.a.q = a.q + row0 * qrow;
+  g.a.out = a.out + row0 * qrow;
+  if (a.out_f32) g.a.out_f32 = a.out_f32 + row0 * qrow;
+  if (a.lse) g.a.lse = a.lse + (size_t)row0 * a.hq;
+  if (a.k_loc) g.a.k_loc = a.k_loc + loc0 * krow;
+  if (a.v_loc) g.a.v_loc = a.v_loc + loc0 * krow;
+  if (a.sel_off) g.a.sel_off = a.sel_off + s0;  // absolute positions in sel_chunk: unchanged
+  if (a.top_ids) g.a.top_ids = a.top_ids + (size_t)s0 * a.top_k;
+}
+
+// More than kMaxSeq sequences: groups of kMaxSeq, run in order on the stream
+// with one workspace, sized for the largest group's need.
+size_t attend_workspace_all(const msa_attend_args& a) {
+  if (a.n_seq <= kMaxSeq) return attend_workspace(a, nullptr);
+  size_t need = 0;
+  AttendGroup g;
+  for (int s0 = 0; s0 < a.n_seq; s0 += kMaxSeq) {
+    attend_group(a, s0, std::min(a.n_seq, s0 + kMaxSeq), g);
+    need = std::max(need, attend_workspace(g.a, nullptr));
+  }
+  return need;
+}
+
+}  // namespace
+
 msa_status msa_attend_workspace(const msa_attend_args* a, size_t* bytes) {
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
   if (!bytes) return fail(MSA_ERR_INVALID_ARG, "attend_workspace: bytes is NULL");
-  *bytes = attend_workspace(*a, nullptr);
+  *bytes = attend_workspace_all(*a);
   return MSA_OK;
 }
 
 msa_status msa_attend(const msa_attend_args* a, void* ws, size_t ws_bytes, void* stream) {
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
-  size_t need = attend_workspace(*a, nullptr);
+  size_t need = attend_workspace_all(*a);
   if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "attend: workspace %zu B, need %zu B", ws_bytes, need);
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(MSA_ERR_WORKSPACE, "attend: workspace must be 256-byte aligned");
   if (a->n_q == 0) return MSA_OK;
-  return launch_attend(*a, ws, (cudaStream_t)stream);
+  if (a->n_seq <= kMaxSeq) return launch_attend(*a, ws, (cudaStream_t)stream);
+  AttendGroup g;
+  for (int s0 = 0; s0 < a->n_seq; s0 += kMaxSeq) {
+    attend_group(*a, s0, std::min(a->n_seq, s0 + kMaxSeq), g);
+    if (g.a.n_q == 0) continue;
+    s = launch_attend(g.a, ws, (cudaStream_t)stream);
+    if (s != MSA_OK) return s;
+  }
+  return MSA_OK;
 }
 
 // ---------------------------------------------------------------- backward
@@ -432,6 +524,7 @@ msa_status msa_attend_backward_workspace(const msa_attend_args* a, size_t* bytes
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
   if (a->top_ids) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: needs a gather listing (sel_off), not the routed form");
+  if (a->n_seq > kMaxSeq) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: n_seq = %d (1..%d)", a->n_seq, kMaxSeq);
   if (!bytes) return fail(MSA_ERR_INVALID_ARG, "attend_backward_workspace: bytes is NULL");
   *bytes = attend_backward_workspace(*a);
   return MSA_OK;
@@ -442,6 +535,7 @@ msa_status msa_attend_backward(const msa_attend_args* a, const float* dout, floa
   msa_status s = check_attend(a);
   if (s != MSA_OK) return s;
   if (a->top_ids) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: needs a gather listing (sel_off), not the routed form");
+  if (a->n_seq > kMaxSeq) return fail(MSA_ERR_UNSUPPORTED, "attend_backward: n_seq = %d (1..%d)", a->n_seq, kMaxSeq);
   if (!a->out_f32 || !a->lse) return fail(MSA_ERR_INVALID_ARG, "attend_backward: the forward's out_f32 and lse are required");
   if (!dout || !dq) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dout or dq");
   if (a->loc_off[a->n_seq] > 0 && (!dk_loc || !dv_loc)) return fail(MSA_ERR_INVALID_ARG, "attend_backward: NULL dk_loc/dv_loc");

@@ -68,7 +68,6 @@ ROUTE_CASES = [
     (dict(kbar_r=None), {}, INVALID, "routing arrays"),
     (dict(kr_inv_norm=None), {}, INVALID, "routing arrays"),
     ({}, dict(n_seq=0), UNSUPPORTED, "n_seq = 0"),
-    ({}, dict(n_seq=257), UNSUPPORTED, "n_seq = 257"),
     ({}, dict(top_k=0), INVALID, "top_k = 0"),
     (dict(n_docs=10000), dict(top_k=5000), UNSUPPORTED, "> 4096"),
     ({}, dict(qr=None), INVALID, "NULL pointer"),
@@ -195,7 +194,6 @@ ATTEND_CASES = [
     (dict(hq=48, hkv=8), UNSUPPORTED, "hq / hkv = 6"),
     (dict(hq=256, hkv=8), UNSUPPORTED, "hq / hkv = 32"),
     (dict(n_seq=0), UNSUPPORTED, "n_seq = 0"),
-    (dict(n_seq=300), UNSUPPORTED, "n_seq = 300"),
     (dict(q=None), INVALID, "NULL pointer"),
     (dict(out=None), INVALID, "NULL pointer"),
     (dict(q_seq_off=[0, 2]), INVALID, "end at n_q"),
@@ -243,6 +241,34 @@ def test_attend_valid_arguments_need_a_workspace(msa):
     # no query rows: nothing to do, nothing enqueued
     z, keep2 = _attend(msa, q_seq_off=[0, 0], n_q=0)
     assert msa._lib.msa_attend(ctypes.byref(z), FAKE, 1 << 30, None) == 0
+
+
+@host_only
+def test_more_than_256_sequences_are_served_in_groups(msa):
+    """Route and attention take any number of sequences (groups of 256 run in
+    turn); their argument checks cover every sequence; the attention backward
+    stays at 256."""
+    S = 300
+    qso = np.arange(S + 1, dtype=np.int32)
+    b = _bank(msa)
+    n = ctypes.c_size_t()
+    n256 = ctypes.c_size_t()
+    assert msa._lib.msa_route_workspace(ctypes.byref(b), S, S, 16, ctypes.byref(n)) == 0
+    assert msa._lib.msa_route_workspace(ctypes.byref(b), 256, S, 16, ctypes.byref(n256)) == 0
+    assert n.value == n256.value  # one group's layout
+    bad = qso.copy()
+    bad[271] = bad[270]  # sequence 270 has no rows: found before anything is enqueued
+    assert msa._lib.msa_route(ctypes.byref(b), FAKE, bad.ctypes.data, S, S, 16, ctypes.c_float(1e-8), FAKE, FAKE,
+                              None, FAKE, 1 << 30, None) == INVALID
+    assert "sequence 270" in _last(msa)
+    a, keep2 = _attend(msa, q_seq_off=qso, q_start=np.zeros(S, np.int32), loc_off=qso, n_seq=S, n_q=S)
+    assert msa._lib.msa_attend_workspace(ctypes.byref(a), ctypes.byref(n)) == 0 and n.value > 0
+    assert msa._lib.msa_attend_backward_workspace(ctypes.byref(a), ctypes.byref(n)) == UNSUPPORTED
+    assert "n_seq = 300" in _last(msa)
+    neg, keep3 = _attend(msa, q_seq_off=qso, q_start=np.r_[np.zeros(280), -1, np.zeros(19)].astype(np.int32),
+                         loc_off=qso, n_seq=S, n_q=S)
+    assert msa._lib.msa_attend(ctypes.byref(neg), FAKE, 1 << 30, None) == INVALID
+    assert "q_start[280]" in _last(msa)
 
 
 @host_only

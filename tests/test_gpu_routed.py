@@ -13,7 +13,7 @@ import pytest
 
 import oracle
 import synth
-from tests.gpu_common import DevBank, bits, from_bits, host_normal, route_gpu
+from tests.gpu_common import DevBank, bits, check_topk, from_bits, host_normal, route_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -175,3 +175,47 @@ def test_tiny_step_route_then_routed_attend(msa):
     msa.sync_check()
     o_out, _ = oracle.attend(q, [0, T], [0], kl, vl, [0, T], kh, vh, o_off, o_sel, pos_offset=16.0)
     assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+
+
+def test_more_than_256_sequences(msa):
+    """300 sequences: the route and the attention run as two groups (256 + 44)
+    on one stream and one workspace each; the top-k against the oracle, the
+    gather listing for all 300 sequences, and the attention (routed form, one
+    decoding row per sequence after 5 local keys) against the oracle chain."""
+    S, L = 300, 5
+    w = synth.workload("tiny")
+    bank = DevBank(w.doc_tok_off, 3, content=True)
+    qr, qso, plan = synth.make_routing_queries(bank.host_chunk_kbar_r, bank.dco, [1] * S, 16, 1, 8, 128, 3)
+    ids, sc, alls = route_gpu(bank, qr, qso, 16)
+    o_ids, o_sc, o_all = oracle.route(bank.host_kbar_r(), bank.dco, qr, qso, 16)
+    check_topk(ids, sc, o_ids, o_sc, o_all)
+    finite = np.isfinite(o_all)
+    np.testing.assert_allclose(alls[finite], o_all[finite], atol=1e-3, rtol=0)
+    top_d = torch.from_numpy(ids).cuda()
+    # the gather listing of all 300 sequences
+    cap = S * 16 * bank.layer_c.max_doc_chunks
+    sel_off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    sel = torch.empty(cap, dtype=torch.int64, device="cuda")
+    msa.gather(bank.layer_c, top_d, 16, sel_off, sel)
+    msa.sync_check()
+    o_off, o_sel = oracle.gather(ids, bank.dco)
+    np.testing.assert_array_equal(sel_off.cpu().numpy(), o_off)
+    np.testing.assert_array_equal(sel.cpu().numpy()[:o_off[-1]], o_sel)
+    # the attention in the routed form
+    q = host_normal((S, 32, 128), synth.tid("q_att", 3))
+    kl = host_normal((S * L, 8, 128), synth.tid("k_loc", 3))
+    vl = host_normal((S * L, 8, 128), synth.tid("v_loc", 3))
+    qs, qst, lo = np.arange(S + 1), np.full(S, L - 1), np.arange(S + 1) * L
+    r = (top_d, bank.layer_c.doc_chunk_off)
+    args = (from_bits(q), qs, qst, from_bits(kl), from_bits(vl), lo, bank.kbar, bank.vbar, None, None,
+            16 * bank.layer_c.max_doc_chunks)
+    out = torch.empty((S, 32, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((S, 32, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((S, 32), dtype=torch.float32, device="cuda")
+    ws = torch.empty(msa.attend_workspace(*args, routed=r), dtype=torch.uint8, device="cuda")
+    msa.attend(*args, out, ws, out_f32=of, lse=lse, pos_offset=16.0, routed=r)
+    msa.sync_check()
+    kh, vh = bank.host_content()
+    o_out, o_lse = oracle.attend(q, qs, qst, kl, vl, lo, kh, vh, o_off, o_sel, pos_offset=16.0)
+    assert np.abs(of.cpu().numpy() - o_out).max() <= 1e-2
+    np.testing.assert_allclose(lse.cpu().numpy(), o_lse, atol=1e-3, rtol=0)
