@@ -49,6 +49,9 @@ def parse_args():
                    help="force the split-K attention's key splits (0: planned)")
     p.add_argument("--gather", choices=["copy", "pull"], default="pull",
                    help="host content tier: copy engine (cudaMemcpyAsync on a side stream) or device pull")
+    p.add_argument("--dec-bulk", type=int, default=-1, choices=[-1, 0, 1],
+                   help="decoding attention: rows by bulk copies (1) or 16-byte cp.async pieces (0); -1: the "
+                        "library's default")
     p.add_argument("--tc-split-blocks", type=int, default=0,
                    help="many-row attention: fewest 64-key blocks per key split (0: the library's plan)")
     p.add_argument("--topk-part", type=int, default=0,
@@ -927,6 +930,8 @@ def config_of(w, eng, args, extra=None):
             cfg["topk_part"] = args.topk_part
         if args.tc_split_blocks:
             cfg["tc_split_blocks"] = args.tc_split_blocks
+        if args.dec_bulk >= 0:
+            cfg["dec_bulk"] = args.dec_bulk
     else:
         cfg.update({"hkv": w.hkv, "tokens_per_doc": 4096})
     cfg["l2"] = "inputs larger than L2 (every step streams all layers' banks)"
@@ -995,6 +1000,8 @@ def run_ours(args):
         msa.set_topk_part(args.topk_part)
     if args.tc_split_blocks:
         msa.set_tc_split_blocks(args.tc_split_blocks)
+    if args.dec_bulk >= 0:
+        msa.set_dec_bulk(bool(args.dec_bulk))
     w = synth.workload(args.workload)
     if args.seqs:
         w.n_seq = args.seqs

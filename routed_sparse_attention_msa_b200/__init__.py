@@ -88,6 +88,7 @@ _sig("msa_debug_set_attend_kernel", [ctypes.c_int])
 _sig("msa_debug_set_attend_splits", [ctypes.c_int])
 _sig("msa_debug_set_topk_part", [ctypes.c_int])
 _sig("msa_debug_set_tc_split_blocks", [ctypes.c_int])
+_sig("msa_debug_set_dec_bulk", [ctypes.c_int])
 _sig("msa_debug_set_dec_rot_keys", [ctypes.c_int])
 _sig("msa_debug_tc_available", [])
 _sig("msa_debug_launch_count", [], ctypes.c_longlong)
@@ -171,6 +172,13 @@ def set_attend_splits(n: int) -> int:
     the previous setting. Workspace sizes follow it: query attend_workspace
     after changing it. Benchmarking control."""
     return int(_lib.msa_debug_set_attend_splits(int(n)))
+
+
+def set_dec_bulk(on: bool) -> bool:
+    """Move the decoding attention kernel's rows by bulk copies (True) or by
+    16-byte cp.async pieces (False); returns the previous setting. Testing
+    control."""
+    return bool(_lib.msa_debug_set_dec_bulk(1 if on else 0))
 
 
 def set_tc_split_blocks(n: int) -> int:

@@ -43,6 +43,7 @@
 #include <math.h>
 
 #include "attend_params.cuh"
+#include "tc_ptx.cuh"
 
 namespace msa {
 namespace {
@@ -142,11 +143,23 @@ __device__ __forceinline__ void rope_pair(float x0, float x1, double pos, double
   y1 = x0 * sn + x1 * cs;
 }
 
+// One 256-byte row by the bulk-copy engine, its bytes counted on the stage's mbarrier.
+__device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 256, [%2];"
+               ::"r"(dst), "l"(src), "r"(bar) : "memory");
+}
+
+// BULK: each of lanes 0-15 moves its own key's rows with one bulk copy per row
+// (completion counted on the warp's stage mbarrier) instead of the warp moving
+// every row in 16-byte cp.async pieces.
+template <bool BULK>
 __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ int64_t s_pre[kDecRoutedMaxK + 1];  // routed form: first list position of each document
   __shared__ int64_t s_c0[kDecRoutedMaxK];       // ... and its first chunk
   __shared__ int64_t s_wsum[kDWarps];
+  __shared__ uint64_t s_bar[kDWarps][2];  // BULK: each warp's two stages
+  __shared__ int s_abort;
   __shared__ double s_invf[kHeadDim / 2];         // RoPE frequency of each pair
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -165,6 +178,15 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   const int ga = g < nvec ? g0 + g / p.group : -1;
   const int gb = g + 8 < nvec ? g0 + (g + 8) / p.group : -1;
 
+  if constexpr (BULK) {
+    if (tid == 0) s_abort = 0;
+    if (lane == 0) {
+      tc::mbar_init(tc::smem_u32(&s_bar[w][0]), 1);
+      tc::mbar_init(tc::smem_u32(&s_bar[w][1]), 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+  }
   pdl_wait();  // the selection comes from an earlier kernel
   pdl_trigger();
 
@@ -270,6 +292,42 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   // k_in_place: the step's local keys are rotated straight into the stage (the warp's first two
   // steps in the in-kernel rotation mode, which has at most 16 local steps), so only V is copied
   auto issue = [&](int i, int64_t r_mine, int stage, bool k_in_place) {
+    if constexpr (BULK) {
+      if (i < nsteps) {
+        uint8_t* stg = wst + stage * kStageB;
+        const bool loc = i < nsl;
+        const uint32_t bar = tc::smem_u32(&s_bar[w][stage]);
+        const int rows = (loc ? (k_in_place ? 1 : 3) : 2);  // 256-byte rows per valid key
+        const unsigned vm = __ballot_sync(0xffffffffu, lane < kStepKeys && r_mine >= 0);
+        if (lane == 0) tc::mbar_expect_tx(bar, (uint32_t)(__popc(vm) * rows * 256));
+        __syncwarp();
+        if (lane < kStepKeys) {
+          const int so = lane * kRowB;
+          if (r_mine >= 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (!loc) {
+              const size_t off = ((size_t)r_mine * row_stride + (size_t)kvh * kHeadDim) * 2;
+              bulk_row(saddr(stg + offSK + so), reinterpret_cast<const uint8_t*>(p.mem_k) + off, bar);
+              bulk_row(saddr(stg + offSV + so), reinterpret_cast<const uint8_t*>(p.mem_v) + off, bar);
+            } else {
+              const size_t lrow = (size_t)(p.loc_off[s] + r_mine) * p.hkv + kvh;
+              if (!k_in_place) {  // rotated by rope_rows: high, then low halves
+                const uint8_t* kr = reinterpret_cast<const uint8_t*>(p.krot) + lrow * kLocRowB;
+                bulk_row(saddr(stg + offSK + so), kr, bar);
+                bulk_row(saddr(stg + offSL + so), kr + 256, bar);
+              }
+              bulk_row(saddr(stg + offSV + so), p.v_loc + lrow * kHeadDim, bar);
+            }
+          } else {
+            // a key past the range: zero values (P is 0 there, and 0 x NaN would not be)
+            uint4* z = reinterpret_cast<uint4*>(stg + offSV + so);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) z[u] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      return;
+    }
     if (i < nsteps) {
       uint8_t* stg = wst + stage * kStageB;
       const bool loc = i < nsl;
@@ -391,7 +449,13 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   int it = 0;
   for (int i = w; i < nsteps; i += kDWarps, ++it) {
     const int stage = it & 1;
-    cp_wait<1>();  // this step's copies (this lane's); the next step's may still be in flight
+    if constexpr (BULK) {  // this step's rows (the next step's may still be in flight)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&s_bar[w][stage]), (uint32_t)((it >> 1) & 1),
+                                                 &s_abort)))
+        break;
+    } else {
+      cp_wait<1>();  // this step's copies (this lane's); the next step's may still be in flight
+    }
     __syncwarp();  // ... and every lane's
     const uint8_t* stg = wst + stage * kStageB;
     const bool loc = i < nsl;
@@ -489,7 +553,7 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
     issue(i + 2 * kDWarps, r_next, stage, false);
     r_next = row_of(i + 3 * kDWarps);
   }
-  cp_wait<0>();
+  if constexpr (!BULK) cp_wait<0>();
   __syncthreads();  // every warp is done with its stages: they hold the merge now
 
   // ---- merge the 8 warps: o [w][v][d], m and l [w][v]
@@ -588,11 +652,10 @@ __global__ void __launch_bounds__(kDThreads, 1) attend_dec_kernel(const __grid_c
   cluster_sync();
 }
 
-}  // namespace
-
-msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st) {
+template <bool BULK>
+msa_status launch_dec(const AttnParams& P, cudaStream_t st) {
   static std::atomic<uint64_t> attr{0};
-  cudaError_t e = smem_limit_once(attend_dec_kernel, kDecSmem, attr);
+  cudaError_t e = smem_limit_once(attend_dec_kernel<BULK>, kDecSmem, attr);
   if (e != cudaSuccess) return cuda_fail(e, "attend: decoding kernel shared memory");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)P.n_splits, (unsigned)P.hkv, (unsigned)P.n_tiles);
@@ -608,9 +671,36 @@ msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st) {
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = P.n_splits > 1 ? 2 : 1;
-  e = cudaLaunchKernelEx(&cfg, attend_dec_kernel, P);
+  e = cudaLaunchKernelEx(&cfg, attend_dec_kernel<BULK>, P);
   if (e != cudaSuccess) return cuda_fail(e, "attend: decoding kernel");
   return launch_check("attend: decoding kernel");
 }
 
+}  // namespace
+
+int g_dec_bulk = 0;  // testing control: the decoding kernel's rows by bulk copies
+
+msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st) {
+  return g_dec_bulk ? launch_dec<true>(P, st) : launch_dec<false>(P, st);
+}
+
+int attend_dec_error_take() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof v) != cudaSuccess) return 0;
+  if (v) {
+    int z = 0;
+    cudaMemcpyToSymbol(g_tc_error, &z, sizeof z);
+  }
+  return v;
+}
+
 }  // namespace msa
+
+// Moves the decoding attention kernel's rows by bulk copies (1) or by 16-byte
+// cp.async pieces (0, the default) in later msa_attend calls; returns the
+// previous setting. A testing and benchmarking control; not declared in msa.h.
+extern "C" int msa_debug_set_dec_bulk(int on) {
+  const int old = msa::g_dec_bulk;
+  if (on == 0 || on == 1) msa::g_dec_bulk = on;
+  return old;
+}

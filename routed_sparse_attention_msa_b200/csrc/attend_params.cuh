@@ -82,6 +82,7 @@ constexpr int kDecMaxSplits = 8;
 constexpr int kDecRoutedMaxK = 256;
 constexpr int kDecRotKeysMax = 256;  // in-kernel rotation: the local keys of a CTA's first 16 steps at most
 msa_status launch_attend_dec(const AttnParams& P, cudaStream_t st);
+int attend_dec_error_take();  // 1 if its bounded wait (bulk-copy rows) ran out since the last call
 int attend_dec_tc_error_take();
 
 }  // namespace msa

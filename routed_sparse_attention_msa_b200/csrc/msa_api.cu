@@ -557,7 +557,7 @@ msa_status msa_sync_check(void* stream) {
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sync_check");
   const int e_tc = tc_error_take(), e_pf = pf_error_take(), e_pr = probe_error_take();
-  const int e_at = attend_tc_error_take() | attend_dec_tc_error_take();
+  const int e_at = attend_tc_error_take() | attend_dec_tc_error_take() | attend_dec_error_take();
   if (e_tc || e_pf) return fail(MSA_ERR_TIMEOUT, "sync_check: a tensor-core scoring kernel gave up on a wait");
   if (e_pr) return fail(MSA_ERR_TIMEOUT, "sync_check: the wait probe's wait ran out");
   if (e_at) return fail(MSA_ERR_TIMEOUT, "sync_check: the tensor-core attention kernel gave up on a wait");

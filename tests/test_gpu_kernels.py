@@ -367,13 +367,16 @@ def test_gather_host_tier(msa, mode):
 
 # ---------------------------------------------------------------- attend
 
-@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope", "dec_bulk"])
 def attend_kernel(request, msa):
     """dec: the decoding kernel rotating its local keys itself; dec_rope: the
-    same kernel after the separate rotation kernel."""
-    old = msa.set_attend_kernel(request.param.replace("_rope", ""))
+    same kernel after the separate rotation kernel; dec_bulk: the decoding
+    kernel moving its rows by bulk copies."""
+    old = msa.set_attend_kernel(request.param.split("_")[0] if request.param.startswith("dec") else request.param)
     old_r = msa.set_dec_rot_keys(0 if request.param == "dec_rope" else 256)
+    old_b = msa.set_dec_bulk(request.param == "dec_bulk")
     yield request.param
+    msa.set_dec_bulk(old_b)
     msa.set_dec_rot_keys(old_r)
     msa.set_attend_kernel(old)
 
@@ -457,7 +460,7 @@ def test_attend_staged_memory_equals_indexed(msa, attend_kernel):
     np.testing.assert_array_equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("kernel", ["split", "dec", "dec_rope"])
+@pytest.mark.parametrize("kernel", ["split", "dec", "dec_rope", "dec_bulk"])
 @pytest.mark.parametrize("splits", [1, 2, 5, 64])
 def test_attend_forced_splits(msa, kernel, splits):
     """Key splits forced (split-K: 64 is clamped to one split per 32 keys;
@@ -465,12 +468,14 @@ def test_attend_forced_splits(msa, kernel, splits):
     walks every key of its sequence): splits that get no keys, one split,
     uneven splits; the decoding kernel rotating its local keys itself or after
     the separate rotation kernel."""
-    old_k, old_s = msa.set_attend_kernel(kernel.replace("_rope", "")), msa.set_attend_splits(splits)
+    old_k, old_s = msa.set_attend_kernel(kernel.split("_")[0]), msa.set_attend_splits(splits)
     old_r = msa.set_dec_rot_keys(0 if kernel == "dec_rope" else 256)
+    old_b = msa.set_dec_bulk(kernel == "dec_bulk")
     try:
         c = _attend_case(rows=(1, 1, 2), n_loc=(65, 1, 9), n_mem=(0, 300, 61), q_start=(64, 0, 7), layer=23)
         g_out, g_f32, g_lse = _attend_gpu(msa, c, 16.0)
     finally:
+        msa.set_dec_bulk(old_b)
         msa.set_dec_rot_keys(old_r)
         msa.set_attend_splits(old_s)
         msa.set_attend_kernel(old_k)

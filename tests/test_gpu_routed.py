@@ -26,13 +26,16 @@ def msa():
     return m
 
 
-@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope"])
+@pytest.fixture(params=["split", "tc", "tc_dec", "dec", "dec_rope", "dec_bulk"])
 def attend_kernel(request, msa):
     """dec: the decoding kernel rotating its local keys itself; dec_rope: the
-    same kernel after the separate rotation kernel."""
-    old = msa.set_attend_kernel(request.param.replace("_rope", ""))
+    same kernel after the separate rotation kernel; dec_bulk: the decoding
+    kernel moving its rows by bulk copies."""
+    old = msa.set_attend_kernel(request.param.split("_")[0] if request.param.startswith("dec") else request.param)
     old_r = msa.set_dec_rot_keys(0 if request.param == "dec_rope" else 256)
+    old_b = msa.set_dec_bulk(request.param == "dec_bulk")
     yield request.param
+    msa.set_dec_bulk(old_b)
     msa.set_dec_rot_keys(old_r)
     msa.set_attend_kernel(old)
 
