@@ -265,6 +265,19 @@ def test_more_than_256_sequences_are_served_in_groups(msa):
     assert msa._lib.msa_attend_workspace(ctypes.byref(a), ctypes.byref(n)) == 0 and n.value > 0
     assert msa._lib.msa_attend_backward_workspace(ctypes.byref(a), ctypes.byref(n)) == UNSUPPORTED
     assert "n_seq = 300" in _last(msa)
+    # the workspace of the whole call is the larger of its two groups' (256 and 44 sequences, the
+    # second with longer local contexts so that it needs more)
+    lo = np.r_[np.arange(257) * 2, 512 + np.arange(1, 45) * 60].astype(np.int32)
+    whole, k4 = _attend(msa, q_seq_off=qso, q_start=np.r_[np.ones(256), np.full(44, 59)].astype(np.int32),
+                        loc_off=lo, n_seq=S, n_q=S)
+    g1, k5 = _attend(msa, q_seq_off=qso[:257], q_start=np.ones(256, np.int32), loc_off=lo[:257], n_seq=256, n_q=256)
+    g2, k6 = _attend(msa, q_seq_off=qso[256:] - 256, q_start=np.full(44, 59, np.int32), loc_off=lo[256:] - lo[256],
+                     n_seq=44, n_q=44)
+    sizes = []
+    for a_ in (whole, g1, g2):
+        assert msa._lib.msa_attend_workspace(ctypes.byref(a_), ctypes.byref(n)) == 0
+        sizes.append(n.value)
+    assert sizes[0] == max(sizes[1], sizes[2]) and sizes[1] != sizes[2]
     neg, keep3 = _attend(msa, q_seq_off=qso, q_start=np.r_[np.zeros(280), -1, np.zeros(19)].astype(np.int32),
                          loc_off=qso, n_seq=S, n_q=S)
     assert msa._lib.msa_attend(ctypes.byref(neg), FAKE, 1 << 30, None) == INVALID
