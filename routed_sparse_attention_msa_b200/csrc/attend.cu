@@ -1018,10 +1018,12 @@ extern "C" int msa_debug_set_attend_kernel(int which) {
   return old;
 }
 
-// Forces the number of key splits of the split-K forward kernel in later
-// msa_attend calls (clamped to 1..64 and to one split per 32 keys); 0 restores
-// the planned count. Returns the previous setting. Workspace sizes follow the
-// setting, so query msa_attend_workspace after changing it. A benchmarking
+// Forces the number of key splits of the forward kernels in later msa_attend
+// calls (split-K kernel: clamped to 1..64 and to one split per 32 keys; the
+// decoding and tensor-core kernels, whose splits form one cluster: to 1..8
+// and to their key blocks); 0 restores the planned count. Returns the
+// previous setting. Workspace sizes follow the setting, so query
+// msa_attend_workspace after changing it. A testing and benchmarking
 // control; not declared in msa.h.
 extern "C" int msa_debug_set_attend_splits(int n) {
   const int old = msa::g_attend_splits;
